@@ -1,0 +1,245 @@
+/*
+ * moe.h — C ABI of the B200 (sm_100a) MoE expert-layer library (libmoe.so).
+ *
+ * The layer: top-k routing of each token to experts, or replay of routing
+ * captured at inference; a stable dispatch of the routed copies grouped by
+ * expert; block-scaled FP8 (e4m3) quantisation in the DeepSeek-V3 style;
+ * grouped FP8 GEMMs of the SiLU-gated expert FFN; a weighted combine; and the
+ * backward of all of it.
+ *
+ * Sources (page titles and sections of the material this library follows):
+ *  [P1] "prime-rl 0.6.0 løfter trillion-parameter RL på lange SWE-flow",
+ *       §Drift og omkostninger i realiteten — each token activates a top-k set
+ *       of experts; dispatch/combine happen in every layer.
+ *  [P4] "RL at 1T scale: prime-rl performance deep dive" —
+ *       §Router Replay: routing decisions made at inference are captured and
+ *       replayed in the trainer; the payload has shape
+ *       [num_layers, top_k, seq_len] and is handled as an opaque tensor;
+ *       §Wide Expert Parallelism, §Parallelism/EP: per-layer dispatch and
+ *       combine of tokens to experts;
+ *       §FP8 Training: block-scaled FP8 as proposed by DeepSeek-V3.
+ *
+ * Conventions (all entry points):
+ *  - Every pointer argument is caller-owned DEVICE memory unless stated; the
+ *    library allocates nothing.  bf16 tensors are passed as uint16_t bit
+ *    patterns.  All matrices are row-major.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default).
+ *  - Calls are asynchronous on `stream` and return a moe_status for the
+ *    host-side checks (arguments, launch).  Errors found on the device
+ *    (bad replay entries, timeouts) are latched in a per-device status word
+ *    read by moe_get_status().
+ *  - No call aborts the process or throws.
+ *
+ * Data layouts (T tokens, D model dim, I expert FFN dim, E experts, k top-k):
+ *  - routed entry i = t*k + j (token t, slot j);
+ *  - R_cap = moe_rows_capacity(dims): bound on the permuted (padded) rows;
+ *    every permuted-row buffer has R_cap rows;
+ *  - 1x128 FP8 of a [rows, C] matrix: codes [rows][C]; scales "K-block
+ *    major" [C/128][ld_rows] (scale of row r, column block b at b*ld_rows+r);
+ *  - 128x1 FP8 (blocks of 128 rows in one column) of a [rows, C] matrix is
+ *    stored transposed: codes [C][ld_rows], scales [ld_rows/128][C];
+ *  - 128x128 FP8 of a weight [N, K]: codes [N][K], scales [N/128][K/128].
+ *  - Scale of a block = fp32(amax / 448) (IEEE fp32 division); code =
+ *    e4m3fn(round-nearest-even, saturate to +-448)(fp32(x / scale));
+ *    a block with amax 0 has scale 0 and codes 0x00.
+ */
+#ifndef MOE_H
+#define MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1, /* null pointer, bad size, misaligned pointer */
+    MOE_ERR_UNSUPPORTED = 2, /* D or I not a multiple of 128, E > 256, k > E, k > 16 */
+    MOE_ERR_CUDA = 3,        /* a CUDA call or launch failed */
+    MOE_ERR_BAD_ROUTING = 4, /* device: replay/permute saw an expert outside [0,E) or a repeat */
+    MOE_ERR_TIMEOUT = 5      /* device: a bounded wait inside a kernel ran out */
+} moe_status;
+
+/* Problem sizes.  align = 1 or 128: each expert's row segment is padded to a
+ * multiple of `align` rows (128 for everything that feeds the GEMMs). */
+typedef struct {
+    int32_t T, D, I, E, k, align;
+} moe_dims;
+
+/* Bound on the permuted rows: T*k + E*(align-1), rounded up to 128. */
+int64_t moe_rows_capacity(const moe_dims *dims);
+
+/* Bytes of caller-provided scratch `ws` for moe_permute. */
+size_t moe_permute_workspace_size(const moe_dims *dims);
+
+const char *moe_strerror(int status);
+
+/* Synchronises `stream`, then reads and clears the device status word of the
+ * current device into *out (MOE_OK if no kernel latched an error). */
+int moe_get_status(void *stream, int *out);
+
+/* Bound (in SM clock cycles) on every spin-wait inside the GEMM kernels;
+ * 0 restores the default (about 2^32 cycles).  On expiry the kernel
+ * latches MOE_ERR_TIMEOUT, drains its own copies and MMAs, frees its tensor
+ * memory and returns. */
+void moe_set_wait_budget(uint64_t cycles);
+
+/* ------------------------------------------------------------------------ */
+/* a1  Top-k routing  [P1 §Drift og omkostninger i realiteten]               */
+/* ------------------------------------------------------------------------ */
+/* logits fp32 [T][E] -> idx int32 [T][k], w fp32 [T][k].
+ * Chooses the k largest logits (compared as fp32; equal logits: lower expert
+ * index first), slots in descending logit order; w = softmax of the chosen
+ * logits (= softmax over all E renormalised over the chosen set).
+ * Logits may be -inf; NaN is not allowed.  E <= 256, k <= min(E, 16). */
+int moe_route_topk(const float *logits, const moe_dims *dims, int32_t *idx, float *w,
+                   void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* a2  Router replay  [P4 §Router Replay]                                    */
+/* ------------------------------------------------------------------------ */
+/* payload int32 [L][k][T] (element (l,j,t) at (l*k+j)*T+t) ->
+ * idx[t][j] = payload[layer][j][t].  Weights: w_in [T][k] copied when non-NULL,
+ * else softmax of the trainer logits [T][E] over the replayed set.  Exactly
+ * one of w_in / logits must be non-NULL.  An entry outside [0,E) or an expert
+ * repeated within a token latches MOE_ERR_BAD_ROUTING; that token's weights
+ * are 0 and its idx entries are copied as given (moe_permute drops entries
+ * outside [0,E)). */
+int moe_route_replay(const int32_t *payload, int32_t L, int32_t layer, const moe_dims *dims,
+                     const float *w_in, const float *logits, int32_t *idx, float *w,
+                     void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* a3+a4  Permute, with the fused 1x128 quantise-and-dispatch                */
+/*        [P4 §Wide Expert Parallelism, §Parallelism/EP; §FP8 Training]      */
+/* ------------------------------------------------------------------------ */
+/* idx [T][k] ->
+ *   counts [E]        routed entries per expert (the per-expert load);
+ *   offsets [E+1]     offsets[0] = 0, offsets[e+1] = offsets[e] + roundup(counts[e], align);
+ *   pos [T][k]        permuted row of entry i: offsets[e] + #{i' < i : idx[i'] = e}
+ *                     (stable), -1 for an entry outside [0,E);
+ *   src_idx [R_cap]   routed entry i = t*k+j held by each permuted row, -1 for
+ *                     padding rows and rows >= offsets[E].
+ * With x (bf16 [T][D]) non-NULL, also dispatches x in FP8:
+ *   xq [R_cap][D] e4m3, xs [D/128][R_cap] fp32: 1x128 blocks of row pos[t][j]
+ *   are those of x[t]; padding rows get codes 0 and scale 0.
+ *   xqT [D][R_cap], xsT [R_cap/128][D] (both nullable, align must be 128):
+ *   128x1 blocks of the permuted rows, for the weight gradient.
+ * ws: moe_permute_workspace_size() bytes of scratch (16-byte aligned). */
+int moe_permute(const int32_t *idx, const moe_dims *dims, int32_t *counts, int32_t *offsets,
+                int32_t *pos, int32_t *src_idx, const uint16_t *x, uint8_t *xq, float *xs,
+                uint8_t *xqT, float *xsT, void *ws, size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* Block-scaled FP8 quantiser  [P4 §FP8 Training]                            */
+/* ------------------------------------------------------------------------ */
+/* in: bf16 [rows][cols], row stride ld elements (ld % 8 == 0, cols % 16 == 0).
+ * (blk_r, blk_c) = (1,128): q [rows][cols], s [ceil(cols/128)][rows];
+ *                  (128,1): q [cols][rows] (transposed), s [ceil(rows/128)][cols],
+ *                           rows % 16 == 0;
+ *                (128,128): q [rows][cols], s [ceil(rows/128)][ceil(cols/128)], and
+ *                           optionally qT [cols][rows], sT [ceil(cols/128)][ceil(rows/128)]
+ *                           (the quantisation of the transpose; rows % 16 == 0).
+ * Edge blocks cover only the elements that exist. */
+int moe_quant_fp8_block(const uint16_t *in, int64_t rows, int64_t cols, int64_t ld,
+                        int32_t blk_r, int32_t blk_c, uint8_t *q, float *s, uint8_t *qT,
+                        float *sT, void *stream);
+
+/* Expert weights (a5): 128x128 FP8 of W_gate, W_up [E][I][D] and W_down [E][D][I].
+ *   wgu_q [E][2I][D], wgu_s [E][2I/128][D/128]: gate and up interleaved by
+ *        128-row blocks (block 2b = gate rows 128b.., block 2b+1 = up rows 128b..);
+ *   wd_q [E][D][I], wd_s [E][D/128][I/128];
+ *   for the backward (all four nullable together):
+ *   wguT_q [E][D][2I], wguT_s [E][D/128][2I/128]  (transpose of wgu);
+ *   wdT_q [E][I][D],   wdT_s [E][I/128][D/128]    (transpose of wd). */
+int moe_quant_weights(const uint16_t *w_gate, const uint16_t *w_up, const uint16_t *w_down,
+                      const moe_dims *dims, uint8_t *wgu_q, float *wgu_s, uint8_t *wd_q,
+                      float *wd_s, uint8_t *wguT_q, float *wguT_s, uint8_t *wdT_q,
+                      float *wdT_s, void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* a6/a7/b2/b3/b4  Grouped block-scaled FP8 GEMMs on tcgen05  [P4 §FP8 Training] */
+/* ------------------------------------------------------------------------ */
+enum {
+    MOE_GEMM_GATEUP_SILU = 0,    /* a6 */
+    MOE_GEMM_DOWN = 1,           /* a7 */
+    MOE_GEMM_DGRAD_DOWN_SILU = 2,/* b2 */
+    MOE_GEMM_DGRAD_GATEUP = 3,   /* b3 */
+    MOE_GEMM_WGRAD_DOWN = 4,     /* b4 */
+    MOE_GEMM_WGRAD_GATEUP = 5    /* b4 */
+};
+
+/* Operands of moe_grouped_gemm_fp8.  For row r of expert e (offsets[e] <= r <
+ * offsets[e+1]) and 1x128 operand scales sa (K-block major, ld R_cap):
+ *
+ * GATEUP_SILU: a = xq [R_cap][D], sa = xs; b = wgu_q, sb = wgu_s.
+ *   g, u = sum over 128-blocks kb of sa[kb][r] * sb[e][n/128][kb] * (a . b)_kb (fp32);
+ *   h = bf16(silu(g) * u); out_q = hq [R_cap][I] e4m3, out_s = hs [I/128][R_cap]
+ *   (1x128 of h).  Nullable: out_bf16 = h [R_cap][I] bf16;
+ *   aux = gu [R_cap][2I] bf16 (g, u saved in wgu's interleaved column order).
+ * DOWN: a = hq, sa = hs; b = wd_q, sb = wd_s; out_bf16 = Y [R_cap][D] bf16.
+ * DGRAD_DOWN_SILU: a = dYq [R_cap][D], sa = dYs; b = wdT_q, sb = wdT_s;
+ *   aux = gu (saved by GATEUP_SILU);  dH = dY . W_down;
+ *   dg = dH*u*s*(1+g*(1-s)), du = dH*silu(g), s = sigmoid(g);
+ *   out_bf16 = dGU [R_cap][2I] bf16 (interleaved like wgu); out_q = dGUq
+ *   [R_cap][2I] e4m3, out_s = dGUs [2I/128][R_cap] (1x128 of dGU).
+ * DGRAD_GATEUP: a = dGUq, sa = dGUs; b = wguT_q, sb = wguT_s;
+ *   out_bf16 = dX [R_cap][D] bf16 (rows in permuted order).
+ * WGRAD_DOWN:   a = dYqT [D][R_cap], sa = dYsT [R_cap/128][D];
+ *               b = hqT [I][R_cap], sb = hsT [R_cap/128][I];
+ *               out_f32 = dWd [E][D][I] fp32, out += sum over the expert's rows.
+ * WGRAD_GATEUP: a = dGUqT [2I][R_cap], sa = dGUsT [R_cap/128][2I];
+ *               b = xqT [D][R_cap], sb = xsT [R_cap/128][D];
+ *               out_f32 = dWgu [E][2I][D] fp32 (interleaved rows), +=.
+ * All code/matrix pointers must be 16-byte aligned. */
+typedef struct {
+    const uint8_t *a;
+    const float *sa;
+    const uint8_t *b;
+    const float *sb;
+    const uint16_t *aux;
+    uint8_t *out_q;
+    float *out_s;
+    uint16_t *out_bf16;
+    float *out_f32;
+} moe_gemm_args;
+
+int moe_grouped_gemm_fp8(int32_t op, const moe_dims *dims, const int32_t *offsets,
+                         const moe_gemm_args *args, void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* a8  Weighted combine  [P1 §Drift og omkostninger; P4 §Parallelism/EP]     */
+/* ------------------------------------------------------------------------ */
+/* y[t] = bf16( sum_{j=0..k-1} w[t][j] * Y[pos[t][j]] ), fp32, j ascending;
+ * entries with pos < 0 are skipped.  Y [R_cap][D] bf16, y [T][D] bf16. */
+int moe_combine(const uint16_t *Y, const float *w, const int32_t *pos, const moe_dims *dims,
+                uint16_t *y, void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* b1  Combine backward  [P4 §FP8 Training]                                  */
+/* ------------------------------------------------------------------------ */
+/* dy [T][D] bf16, Y [R_cap][D] bf16, w, pos, idx [T][k] ->
+ *   dYq [R_cap][D] e4m3, dYs [D/128][R_cap]: 1x128 of the rows
+ *        dY[pos[t][j]] = bf16(fp32(w[t][j] * dy[t])), padding rows 0;
+ *   dY_bf16 [R_cap][D] (nullable): those rows in bf16;
+ *   d_w [T][k] = <dy[t], Y[pos[t][j]]> (fp32);
+ *   d_logits [T][E] (nullable; w must be the softmax over the chosen set):
+ *        w_j * (d_w_j - sum_i w_i d_w_i) at the chosen experts, 0 elsewhere.
+ * counts and offsets (from moe_permute) locate the padding rows, which are
+ * written as zeros (codes, scales and dY_bf16). */
+int moe_combine_bwd(const uint16_t *dy, const uint16_t *Y, const float *w, const int32_t *pos,
+                    const int32_t *idx, const int32_t *counts, const int32_t *offsets,
+                    const moe_dims *dims,
+                    uint8_t *dYq, float *dYs, uint16_t *dY_bf16, float *d_w, float *d_logits,
+                    void *stream);
+
+/* b3  dx[t] = bf16( sum_j dX[pos[t][j]] ), fp32, j ascending. */
+int moe_unpermute_reduce(const uint16_t *dX, const int32_t *pos, const moe_dims *dims,
+                         uint16_t *dx, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_H */

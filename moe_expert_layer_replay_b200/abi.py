@@ -1,0 +1,176 @@
+"""ctypes binding of libmoe.so: one Python function per C entry point, same
+names without the ``moe_`` prefix.  Argument marshalling only — every step of
+the layer runs in the library's CUDA kernels; torch tensors supply device
+memory and the current stream.  Contracts and layouts: include/moe.h.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libmoe.so")
+
+OK, INVALID_ARG, UNSUPPORTED, CUDA_ERR, BAD_ROUTING, TIMEOUT = range(6)
+GEMM_GATEUP_SILU, GEMM_DOWN, GEMM_DGRAD_DOWN_SILU, GEMM_DGRAD_GATEUP, GEMM_WGRAD_DOWN, GEMM_WGRAD_GATEUP = range(6)
+
+EXPORTS = [
+    "moe_rows_capacity", "moe_permute_workspace_size", "moe_strerror", "moe_get_status",
+    "moe_set_wait_budget", "moe_route_topk", "moe_route_replay", "moe_permute",
+    "moe_quant_fp8_block", "moe_quant_weights", "moe_grouped_gemm_fp8", "moe_combine",
+    "moe_combine_bwd", "moe_unpermute_reduce",
+]
+
+
+class MoeError(RuntimeError):
+    def __init__(self, call: str, status: int):
+        super().__init__(f"{call}: {strerror(status)} (status {status})")
+        self.status = status
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("D", ctypes.c_int32), ("I", ctypes.c_int32),
+                ("E", ctypes.c_int32), ("k", ctypes.c_int32), ("align", ctypes.c_int32)]
+
+    def __repr__(self):
+        return f"Dims(T={self.T}, D={self.D}, I={self.I}, E={self.E}, k={self.k}, align={self.align})"
+
+
+class GemmArgs(ctypes.Structure):
+    _fields_ = [("a", ctypes.c_void_p), ("sa", ctypes.c_void_p), ("b", ctypes.c_void_p),
+                ("sb", ctypes.c_void_p), ("aux", ctypes.c_void_p), ("out_q", ctypes.c_void_p),
+                ("out_s", ctypes.c_void_p), ("out_bf16", ctypes.c_void_p), ("out_f32", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmoe.so.  Raises if it has not been built: there is no fallback."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m moe_expert_layer_replay_b200.build` (nvcc, sm_100a)")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I32, I64, SZ, U64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_uint64
+        D = ctypes.POINTER(Dims)
+        sig = {
+            "moe_rows_capacity": (I64, [D]),
+            "moe_permute_workspace_size": (SZ, [D]),
+            "moe_strerror": (ctypes.c_char_p, [ctypes.c_int]),
+            "moe_get_status": (ctypes.c_int, [P, ctypes.POINTER(ctypes.c_int)]),
+            "moe_set_wait_budget": (None, [U64]),
+            "moe_route_topk": (ctypes.c_int, [P, D, P, P, P]),
+            "moe_route_replay": (ctypes.c_int, [P, I32, I32, D, P, P, P, P, P]),
+            "moe_permute": (ctypes.c_int, [P, D, P, P, P, P, P, P, P, P, P, P, SZ, P]),
+            "moe_quant_fp8_block": (ctypes.c_int, [P, I64, I64, I64, I32, I32, P, P, P, P, P]),
+            "moe_quant_weights": (ctypes.c_int, [P, P, P, D, P, P, P, P, P, P, P, P, P]),
+            "moe_grouped_gemm_fp8": (ctypes.c_int, [I32, D, P, ctypes.POINTER(GemmArgs), P]),
+            "moe_combine": (ctypes.c_int, [P, P, P, D, P, P]),
+            "moe_combine_bwd": (ctypes.c_int, [P, P, P, P, P, P, P, D, P, P, P, P, P, P]),
+            "moe_unpermute_reduce": (ctypes.c_int, [P, P, D, P, P]),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _p(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return ctypes.c_void_p(t)
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _s(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check(name, st):
+    if st != OK:
+        raise MoeError(name, st)
+
+
+def dims(T, D, I, E, k, align=128) -> Dims:
+    return Dims(int(T), int(D), int(I), int(E), int(k), int(align))
+
+
+# ---------------------------------------------------------------- queries --
+def rows_capacity(d: Dims) -> int:
+    return int(lib().moe_rows_capacity(ctypes.byref(d)))
+
+
+def permute_workspace_size(d: Dims) -> int:
+    return int(lib().moe_permute_workspace_size(ctypes.byref(d)))
+
+
+def strerror(st: int) -> str:
+    return lib().moe_strerror(int(st)).decode()
+
+
+def get_status(stream=None) -> int:
+    out = ctypes.c_int(0)
+    _check("moe_get_status", lib().moe_get_status(_s(stream), ctypes.byref(out)))
+    return out.value
+
+
+def set_wait_budget(cycles: int) -> None:
+    lib().moe_set_wait_budget(int(cycles))
+
+
+# ------------------------------------------------------------ entry points --
+def route_topk(logits, d: Dims, idx, w, stream=None):
+    _check("moe_route_topk", lib().moe_route_topk(_p(logits), ctypes.byref(d), _p(idx), _p(w), _s(stream)))
+
+
+def route_replay(payload, L, layer, d: Dims, w_in, logits, idx, w, stream=None):
+    _check("moe_route_replay", lib().moe_route_replay(_p(payload), int(L), int(layer), ctypes.byref(d),
+                                                      _p(w_in), _p(logits), _p(idx), _p(w), _s(stream)))
+
+
+def permute(idx, d: Dims, counts, offsets, pos, src_idx, x, xq, xs, xqT, xsT, ws, stream=None):
+    _check("moe_permute", lib().moe_permute(_p(idx), ctypes.byref(d), _p(counts), _p(offsets), _p(pos),
+                                            _p(src_idx), _p(x), _p(xq), _p(xs), _p(xqT), _p(xsT), _p(ws),
+                                            ws.numel() * ws.element_size(), _s(stream)))
+
+
+def quant_fp8_block(inp, rows, cols, ld, blk_r, blk_c, q, s, qT=None, sT=None, stream=None):
+    _check("moe_quant_fp8_block", lib().moe_quant_fp8_block(_p(inp), int(rows), int(cols), int(ld), int(blk_r),
+                                                            int(blk_c), _p(q), _p(s), _p(qT), _p(sT), _s(stream)))
+
+
+def quant_weights(w_gate, w_up, w_down, d: Dims, wgu_q, wgu_s, wd_q, wd_s,
+                  wguT_q=None, wguT_s=None, wdT_q=None, wdT_s=None, stream=None):
+    _check("moe_quant_weights", lib().moe_quant_weights(_p(w_gate), _p(w_up), _p(w_down), ctypes.byref(d),
+                                                        _p(wgu_q), _p(wgu_s), _p(wd_q), _p(wd_s), _p(wguT_q),
+                                                        _p(wguT_s), _p(wdT_q), _p(wdT_s), _s(stream)))
+
+
+def grouped_gemm_fp8(op, d: Dims, offsets, a, sa, b, sb, aux=None, out_q=None, out_s=None,
+                     out_bf16=None, out_f32=None, stream=None):
+    g = GemmArgs(*[None if t is None else t.data_ptr() for t in (a, sa, b, sb, aux, out_q, out_s, out_bf16, out_f32)])
+    _check("moe_grouped_gemm_fp8", lib().moe_grouped_gemm_fp8(int(op), ctypes.byref(d), _p(offsets),
+                                                              ctypes.byref(g), _s(stream)))
+
+
+def combine(Y, w, pos, d: Dims, y, stream=None):
+    _check("moe_combine", lib().moe_combine(_p(Y), _p(w), _p(pos), ctypes.byref(d), _p(y), _s(stream)))
+
+
+def combine_bwd(dy, Y, w, pos, idx, counts, offsets, d: Dims, dYq, dYs, dY_bf16, d_w, d_logits, stream=None):
+    _check("moe_combine_bwd", lib().moe_combine_bwd(_p(dy), _p(Y), _p(w), _p(pos), _p(idx), _p(counts),
+                                                    _p(offsets), ctypes.byref(d), _p(dYq), _p(dYs), _p(dY_bf16),
+                                                    _p(d_w), _p(d_logits), _s(stream)))
+
+
+def unpermute_reduce(dX, pos, d: Dims, dx, stream=None):
+    _check("moe_unpermute_reduce", lib().moe_unpermute_reduce(_p(dX), _p(pos), ctypes.byref(d), _p(dx), _s(stream)))

@@ -1,0 +1,707 @@
+// Grouped block-scaled FP8 GEMMs of the expert FFN on sm_100a tensor cores
+// (a6 gate/up + SiLU + h-quant, a7 down, b2 dgrad down + SiLU backward,
+// b3 dgrad gate/up, b4 wgrad).  Block-scaled FP8 as proposed by DeepSeek-V3
+// is what the trainer runs ("RL at 1T scale: prime-rl performance deep
+// dive", §FP8 Training).
+//
+// Design (one persistent CTA per SM, 12 warps = 3 warpgroups):
+//   warp 0     TMA producer: 128-byte-swizzled tiles of A (128 x 128 B) and
+//              B (256 x 128 B) per 128-deep K block into a 4-stage ring;
+//   warp 1     allocates 512 TMEM columns; lane 0 issues tcgen05.mma
+//              (kind::f8f6f4, e4m3 x e4m3 -> fp32, M=128, N=256, K=32) x4
+//              per K block into one of two 256-column TMEM accumulators;
+//   warps 2-3  idle (they complete warpgroup 0, which gives its registers
+//              to the epilogue: setmaxnreg 56 here, 224 in warpgroups 1-2;
+//              128*56 + 256*224 = 384*168, the launch allocation);
+//   warps 4-11 epilogue: per K block, read the accumulator with tcgen05.ld,
+//              multiply by that block's scales (row scale x weight-block
+//              scale; per-column for wgrad) and add into fp32 registers; the
+//              freed TMEM buffer is handed back while the MMA fills the
+//              other.  After the last K block: the fused output step.
+// The scales are arbitrary fp32 (amax/448), so they cannot ride in the
+// hardware block-scaled MMA (which takes power-of-two UE8M0 scales); each
+// K block's partial product is promoted in fp32 instead.
+//
+// Tile spaces:
+//   rows mode (a6, a7, b2, b3): one tile = 128 permuted rows (always inside
+//   one expert: segments are 128-aligned) x 256 output columns; K = D, I or
+//   2I.  The number of row tiles, offsets[E]/128, is read on the device.
+//   wgrad mode (b4): one tile = (expert, 128 rows of dW, 256 columns of dW);
+//   K runs over the expert's permuted rows.
+//
+// Every mbarrier wait is bounded; on expiry the kernel latches
+// MOE_ERR_TIMEOUT, drains the copies and MMAs it issued, frees TMEM and exits.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+namespace gemm {
+
+constexpr int BM = 128, BN = 256, BK = 128;
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK, B_BYTES = BN * BK, STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int NUM_THREADS = 384;
+constexpr int EPI_WARP0 = 4;
+constexpr int EPI_THREADS = 256;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint64_t DRAIN_BUDGET = 1ull << 28;
+// smem: ring | barriers (full[4], empty[4], tfull[2], tempty[2], drain, epi) |
+// tmem slot | abort flag | offsets[257] | amax exchange [2][2][128] | wgrad col scales [2][256]
+constexpr int OFF_BAR = STAGES * STAGE_BYTES;
+constexpr int OFF_TMEM_SLOT = OFF_BAR + 16 * 8;
+constexpr int OFF_ABORT = OFF_TMEM_SLOT + 4;
+constexpr int OFF_OFFSETS = OFF_BAR + 256;
+constexpr int OFF_AMAX = OFF_OFFSETS + 1040;
+constexpr int OFF_COLSCALE = OFF_AMAX + 2 * 2 * 128 * 4;
+constexpr int SMEM_BYTES = OFF_COLSCALE + 2 * 256 * 4 + 1024;  // + alignment slack
+
+enum Epi { EPI_SILU = 0, EPI_BF16 = 1, EPI_DSILU = 2, EPI_WGRAD = 3 };
+
+struct Args {
+    const int32_t *offsets;
+    int E;
+    int64_t R_cap;
+    int M;  // wgrad: rows of dW (D or 2I)
+    int N;  // output columns
+    int K;  // rows mode: reduction length
+    const float *sa;
+    const float *sb;
+    const uint16_t *aux;
+    uint8_t *out_q;
+    float *out_s;
+    uint16_t *out_bf16;
+    float *out_f32;
+    int *status;
+    uint64_t budget;
+};
+
+// ----------------------------------------------------------------- PTX ----
+__device__ __forceinline__ uint32_t smem_u32(const void *p)
+{
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.b32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+// Bounded wait.  Returns false when the CTA is aborting (flag set by any role)
+// or when this wait ran out (then it sets the flag and latches the status).
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, uint64_t budget,
+                                             volatile int *abort_flag, int *status)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if ((uint64_t)(clock64() - t0) > budget) {
+            *abort_flag = 1;
+            latch_status(status, MOE_ERR_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+// Drain wait: ignores the abort flag (used on the way out).
+__device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity)
+{
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity))
+        if ((uint64_t)(clock64() - t0) > DRAIN_BUDGET) return;
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int32_t c0,
+                                            int32_t c1, uint32_t bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
+        : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
+// 1024 bytes apart (SBO), version 1 (sm_100), base offset 0 (1024-aligned).
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr)
+{
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+    d |= (uint64_t)1 << 16;             // leading byte offset (unused when swizzled)
+    d |= (uint64_t)(1024 >> 4) << 32;   // stride byte offset
+    d |= (uint64_t)1 << 46;             // descriptor version
+    d |= (uint64_t)2 << 61;             // SWIZZLE_128B
+    return d;
+}
+
+// Instruction descriptor, kind::f8f6f4: D fp32, A and B e4m3, both K-major,
+// N = 256, M = 128.
+constexpr uint32_t IDESC = (1u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                           ((uint32_t)(BM >> 4) << 24);
+
+__device__ __forceinline__ void mma_f8(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t accum)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(a), "l"(b), "r"(IDESC), "r"(accum));
+}
+
+__device__ __forceinline__ void mma_commit(uint32_t bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+
+#define MOE_TMEM_LD32(taddr, r)                                                                        \
+    asm volatile(                                                                                      \
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"   \
+        "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"                 \
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),          \
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),      \
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),   \
+          "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),   \
+          "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])                                           \
+        : "r"(taddr))
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+
+// ------------------------------------------------------------ schedule ----
+struct Tile {
+    int e;      // expert
+    int m0;     // first row (rows mode: permuted row; wgrad: row of dW)
+    int n0;     // first output column
+    int nt;     // column-tile index
+    int kb0;    // first K block
+    int kb1;    // one past the last K block
+};
+
+template <bool kWgrad>
+__device__ __forceinline__ int num_tiles(const Args &p, const int *offs_s)
+{
+    const int NT = (p.N + BN - 1) / BN;
+    if (kWgrad) return p.E * (p.M / BM) * NT;
+    return (offs_s[p.E] / BM) * NT;
+}
+
+template <bool kWgrad>
+__device__ __forceinline__ Tile tile_of(int t, const Args &p, const int *offs_s)
+{
+    const int NT = (p.N + BN - 1) / BN;
+    Tile x;
+    if (kWgrad) {
+        const int MT = p.M / BM;
+        x.e = t / (MT * NT);
+        int rem = t - x.e * MT * NT;
+        int mt = rem / NT;
+        x.nt = rem - mt * NT;
+        x.m0 = mt * BM;
+        x.n0 = x.nt * BN;
+        x.kb0 = offs_s[x.e] / BK;
+        x.kb1 = offs_s[x.e + 1] / BK;
+    } else {
+        int mt = t / NT;
+        x.nt = t - mt * NT;
+        x.m0 = mt * BM;
+        x.n0 = x.nt * BN;
+        int lo = 0, hi = p.E - 1;  // last e with offs[e] <= m0
+        while (lo < hi) {
+            int mid = (lo + hi + 1) >> 1;
+            if (offs_s[mid] <= x.m0) lo = mid; else hi = mid - 1;
+        }
+        x.e = lo;
+        x.kb0 = 0;
+        x.kb1 = p.K / BK;
+    }
+    return x;
+}
+
+// --------------------------------------------------------------- kernel ----
+template <int kEpi>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const Args p)
+{
+    constexpr bool kWgrad = (kEpi == EPI_WGRAD);
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t bar_full = sbase + OFF_BAR;           // [STAGES]
+    const uint32_t bar_empty = bar_full + STAGES * 8;     // [STAGES]
+    const uint32_t bar_tfull = bar_empty + STAGES * 8;    // [2]
+    const uint32_t bar_tempty = bar_tfull + 2 * 8;        // [2]
+    const uint32_t bar_drain = bar_tempty + 2 * 8;
+    const uint32_t bar_epi = bar_drain + 8;  // the 256 epilogue threads meet here
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_ABORT);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_TMEM_SLOT);
+    int *offs_s = reinterpret_cast<int *>(smem + OFF_OFFSETS);
+    float *amax_s = reinterpret_cast<float *>(smem + OFF_AMAX);       // [2][2][128]
+    float *colscale_s = reinterpret_cast<float *>(smem + OFF_COLSCALE);  // [2][256]
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    for (int i = threadIdx.x; i <= p.E; i += blockDim.x) offs_s[i] = p.offsets[i];
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(bar_full + 8 * s, 1);
+            mbar_init(bar_empty + 8 * s, 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bar_tfull + 8 * b, 1);
+            mbar_init(bar_tempty + 8 * b, EPI_THREADS / 32);
+        }
+        mbar_init(bar_drain, 1);
+        mbar_init(bar_epi, EPI_THREADS);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(TMEM_COLS));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int ntiles = num_tiles<kWgrad>(p, offs_s);
+
+    if (warp < EPI_WARP0) {
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 56;");
+      if (warp == 0) {
+        // ------------------------------------------------ TMA producer ----
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t pend = 0, pend_phase = 0;  // loads issued, not yet seen consumed
+            bool ok = true;
+            for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+                const Tile x = tile_of<kWgrad>(t, p, offs_s);
+                for (int kb = x.kb0; kb < x.kb1; ++kb) {
+                    if (!wait_bounded(bar_empty + 8 * stage, phase ^ 1, p.budget, abort_flag, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    pend &= ~(1u << stage);
+                    const uint32_t fb = bar_full + 8 * stage;
+                    const uint32_t dA = sbase + stage * STAGE_BYTES, dB = dA + A_BYTES;
+                    mbar_arrive_expect_tx(fb, STAGE_BYTES);
+                    if (kWgrad) {
+                        tma_load_2d(dA, &tmA, kb * BK, x.m0, fb);
+                        tma_load_2d(dB, &tmB, kb * BK, x.n0, fb);
+                    } else {
+                        tma_load_2d(dA, &tmA, kb * BK, x.m0, fb);
+                        tma_load_2d(dB, &tmB, kb * BK, x.e * p.N + x.n0, fb);
+                    }
+                    pend |= 1u << stage;
+                    pend_phase = (pend_phase & ~(1u << stage)) | (phase << stage);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+            }
+            if (!ok) {
+                for (int s = 0; s < STAGES; ++s)
+                    if (pend & (1u << s)) wait_drain(bar_full + 8 * s, (pend_phase >> s) & 1u);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------- MMA issuer ----
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int buf = 0;
+            uint32_t bphase = 0;
+            bool ok = true, issued = false;
+            for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+                const Tile x = tile_of<kWgrad>(t, p, offs_s);
+                for (int kb = x.kb0; kb < x.kb1; ++kb) {
+                    if (!wait_bounded(bar_tempty + 8 * buf, bphase ^ 1, p.budget, abort_flag, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    if (!wait_bounded(bar_full + 8 * stage, phase, p.budget, abort_flag, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t aA = sbase + stage * STAGE_BYTES, aB = aA + A_BYTES;
+                    const uint32_t dtm = tmem_base + (uint32_t)(buf * BN);
+#pragma unroll
+                    for (int k4 = 0; k4 < BK / 32; ++k4)
+                        mma_f8(dtm, sdesc(aA + 32 * k4), sdesc(aB + 32 * k4), k4 > 0 ? 1u : 0u);
+                    issued = true;
+                    mma_commit(bar_empty + 8 * stage);
+                    mma_commit(bar_tfull + 8 * buf);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                    buf ^= 1;
+                    if (buf == 0) bphase ^= 1;
+                }
+            }
+            if (issued) {
+                mma_commit(bar_drain);
+                wait_drain(bar_drain, 0);
+            }
+        }
+      }
+    } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 224;");
+        // --------------------------------------------------- epilogue ----
+        const int ew = warp - EPI_WARP0;     // 0..7
+        const int q = warp & 3;              // TMEM lane quarter of this warp
+        const int h = ew >> 2;               // column half
+        const int row = 32 * q + lane;       // row within the tile
+        const int et = threadIdx.x - 32 * EPI_WARP0;  // 0..255
+        const uint32_t lane_addr = tmem_base + ((uint32_t)(32 * q) << 16);
+        const int KB = p.K / BK, NB = p.N / BK;
+        int buf = 0;
+        uint32_t bphase = 0;
+        int tcount = 0;
+        bool ok = true;
+        uint32_t ephase = 0;
+        // all epilogue threads meet; bounded, so an aborting CTA cannot hang here
+        auto epi_sync = [&]() -> bool {
+            mbar_arrive(bar_epi);
+            bool r = wait_bounded(bar_epi, ephase, p.budget, abort_flag, p.status);
+            ephase ^= 1;
+            return r;
+        };
+        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++tcount) {
+            const Tile x = tile_of<kWgrad>(t, p, offs_s);
+            if (kWgrad && x.kb1 == x.kb0) continue;
+            float acc[128];
+#pragma unroll
+            for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
+            // scale fetch for K block kb
+            auto fetch = [&](int kb, float &sa, float &s0, float &s1, float &cs) {
+                if (kWgrad) {
+                    sa = p.sa[(int64_t)kb * p.M + x.m0 + row];
+                    const int c = x.n0 + et;
+                    cs = (c < p.N) ? p.sb[(int64_t)kb * p.N + c] : 0.0f;
+                    s0 = s1 = 0.0f;
+                } else {
+                    sa = p.sa[(int64_t)kb * p.R_cap + x.m0 + row];
+                    const int64_t sbrow = (int64_t)x.e * NB + 2 * x.nt;
+                    if (kEpi == EPI_SILU) {
+                        s0 = p.sb[sbrow * KB + kb];        // gate block
+                        s1 = p.sb[(sbrow + 1) * KB + kb];  // up block
+                    } else {
+                        const int64_t nb = sbrow + h;
+                        s0 = s1 = (2 * x.nt + h < NB) ? p.sb[nb * KB + kb] : 0.0f;
+                    }
+                    cs = 0.0f;
+                }
+            };
+            float n_sa, n_s0, n_s1, n_cs;
+            fetch(x.kb0, n_sa, n_s0, n_s1, n_cs);
+            for (int kb = x.kb0; kb < x.kb1; ++kb) {
+                const float sa = n_sa, s0 = n_s0, s1 = n_s1, cs = n_cs;
+                if (kb + 1 < x.kb1) fetch(kb + 1, n_sa, n_s0, n_s1, n_cs);
+                float *cscale = colscale_s + (kb & 1) * 256;
+                if (kWgrad) {
+                    cscale[et] = cs;
+                    if (!epi_sync()) {
+                        ok = false;
+                        break;
+                    }
+                }
+                if (!wait_bounded(bar_tfull + 8 * buf, bphase, p.budget, abort_flag, p.status)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t cbase = lane_addr + (uint32_t)(buf * BN);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t col;
+                    if (kEpi == EPI_SILU) col = (c < 2) ? (64 * h + 32 * c) : (128 + 64 * h + 32 * (c - 2));
+                    else col = 128 * h + 32 * c;
+                    uint32_t r[32];
+                    MOE_TMEM_LD32(cbase + col, r);
+                    tmem_wait_ld();
+                    if (kWgrad) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            acc[32 * c + i] = fmaf(__uint_as_float(r[i]), sa * cscale[col + i], acc[32 * c + i]);
+                    } else {
+                        const float sc = sa * ((kEpi == EPI_SILU && c >= 2) ? s1 : s0);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) acc[32 * c + i] = fmaf(__uint_as_float(r[i]), sc, acc[32 * c + i]);
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_tempty + 8 * buf);
+                buf ^= 1;
+                if (buf == 0) bphase ^= 1;
+            }
+            if (!ok) break;
+            const int64_t r = (int64_t)x.m0 + row;
+            // ------------------------------------------- fused outputs ----
+            if (kEpi == EPI_SILU) {
+                // acc[0..63] = g, acc[64..127] = u of I-columns nt*128 + 64h + i
+                const int64_t I = p.N / 2;
+                const int64_t icol = (int64_t)x.nt * 128 + 64 * h;
+                float amax = 0.0f;
+#pragma unroll
+                for (int i0 = 0; i0 < 64; i0 += 8) {
+                    if (p.aux) {
+                        uint16_t *gu = const_cast<uint16_t *>(p.aux) + r * p.N + x.n0 + 64 * h + i0;
+                        *reinterpret_cast<uint4 *>(gu) = pack8(&acc[i0]);
+                        *reinterpret_cast<uint4 *>(gu + 128) = pack8(&acc[64 + i0]);
+                    }
+#pragma unroll
+                    for (int i = i0; i < i0 + 8; ++i) {
+                        const float g = acc[i], u = acc[64 + i];
+                        const float sg = g / (1.0f + expf(-g));
+                        const float hv = __uint_as_float(bf16_bits_rn(sg * u) << 16);
+                        acc[i] = hv;
+                        amax = fmaxf(amax, fabsf(hv));
+                    }
+                }
+                float *ax = amax_s + (tcount & 1) * 256;
+                ax[h * 128 + row] = amax;
+                if (!epi_sync()) break;
+                amax = fmaxf(ax[row], ax[128 + row]);
+                const float s = block_scale(amax);
+                uint8_t *hq = p.out_q + r * I + icol;
+#pragma unroll
+                for (int i0 = 0; i0 < 64; i0 += 16) *reinterpret_cast<uint4 *>(hq + i0) = quant16(&acc[i0], s);
+                if (h == 0) p.out_s[(int64_t)x.nt * p.R_cap + r] = s;
+                if (p.out_bf16) {
+                    uint16_t *hb = p.out_bf16 + r * I + icol;
+#pragma unroll
+                    for (int i0 = 0; i0 < 64; i0 += 8) *reinterpret_cast<uint4 *>(hb + i0) = pack8(&acc[i0]);
+                }
+            } else if (kEpi == EPI_BF16) {
+                const int64_t c0 = (int64_t)x.n0 + 128 * h;
+                if (c0 < p.N) {
+                    uint16_t *o = p.out_bf16 + r * p.N + c0;
+#pragma unroll
+                    for (int i0 = 0; i0 < 128; i0 += 8) *reinterpret_cast<uint4 *>(o + i0) = pack8(&acc[i0]);
+                }
+            } else if (kEpi == EPI_DSILU) {
+                // acc = dH of I-block nb = 2nt + h; gate/up columns of that block
+                // in the interleaved 2I space: 2nb*128 and (2nb+1)*128
+                const int nb = 2 * x.nt + h;
+                if (nb * 128 < p.N) {
+                    const int64_t N2 = 2 * (int64_t)p.N;
+                    const int64_t gc = (int64_t)(2 * nb) * 128, uc = gc + 128;
+                    const uint16_t *gu = p.aux + r * N2;
+                    float amax_g = 0.0f, amax_u = 0.0f;
+#pragma unroll
+                    for (int i0 = 0; i0 < 128; i0 += 8) {
+                        asm volatile("" ::: "memory");  // keep one chunk's loads live at a time
+                        float g[8], u[8], dg[8], du[8];
+                        unpack8(*reinterpret_cast<const uint4 *>(gu + gc + i0), g);
+                        unpack8(*reinterpret_cast<const uint4 *>(gu + uc + i0), u);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const float dh = acc[i0 + i];
+                            const float sg = 1.0f / (1.0f + expf(-g[i]));
+                            const float dgv = dh * u[i] * sg * (1.0f + g[i] * (1.0f - sg));
+                            const float duv = dh * g[i] * sg;
+                            const uint32_t bg = bf16_bits_rn(dgv), bu = bf16_bits_rn(duv);
+                            dg[i] = __uint_as_float(bg << 16);
+                            du[i] = __uint_as_float(bu << 16);
+                            amax_g = fmaxf(amax_g, fabsf(dg[i]));
+                            amax_u = fmaxf(amax_u, fabsf(du[i]));
+                            acc[i0 + i] = __uint_as_float(bg | (bu << 16));
+                        }
+                        if (p.out_bf16) {
+                            *reinterpret_cast<uint4 *>(p.out_bf16 + r * N2 + gc + i0) = pack8(dg);
+                            *reinterpret_cast<uint4 *>(p.out_bf16 + r * N2 + uc + i0) = pack8(du);
+                        }
+                    }
+                    const float sgs = block_scale(amax_g), sus = block_scale(amax_u);
+#pragma unroll
+                    for (int i0 = 0; i0 < 128; i0 += 16) {
+                        float dg[16], du[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const uint32_t w = __float_as_uint(acc[i0 + i]);
+                            dg[i] = __uint_as_float(w << 16);
+                            du[i] = __uint_as_float(w & 0xffff0000u);
+                        }
+                        *reinterpret_cast<uint4 *>(p.out_q + r * N2 + gc + i0) = quant16(dg, sgs);
+                        *reinterpret_cast<uint4 *>(p.out_q + r * N2 + uc + i0) = quant16(du, sus);
+                    }
+                    p.out_s[(int64_t)(2 * nb) * p.R_cap + r] = sgs;
+                    p.out_s[(int64_t)(2 * nb + 1) * p.R_cap + r] = sus;
+                }
+            } else {  // EPI_WGRAD: dW[e][m][n] += acc
+                const int64_t c0 = (int64_t)x.n0 + 128 * h;
+                if (c0 < p.N) {
+                    float *o = p.out_f32 + ((int64_t)x.e * p.M + x.m0 + row) * p.N + c0;
+#pragma unroll
+                    for (int i0 = 0; i0 < 128; i0 += 4) {
+                        float4 v = *reinterpret_cast<float4 *>(o + i0);
+                        v.x += acc[i0];
+                        v.y += acc[i0 + 1];
+                        v.z += acc[i0 + 2];
+                        v.w += acc[i0 + 3];
+                        *reinterpret_cast<float4 *>(o + i0) = v;
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS));
+}
+
+}  // namespace gemm
+
+// ------------------------------------------------------------------ host ----
+static PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void *ptr = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// 2D uint8 tensor [rows][cols] (row stride cols bytes), box box_rows x 128
+// bytes, 128-byte swizzle; out-of-range elements read as zero.
+static bool make_map(CUtensorMap *map, const void *base, uint64_t cols, uint64_t rows, uint32_t box_rows)
+{
+    auto fn = get_encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols};
+    cuuint32_t box[2] = {128, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+static int sm_count()
+{
+    int dev = 0, n = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 148;
+}
+
+template <int kEpi>
+static int launch_one(const CUtensorMap &a, const CUtensorMap &b, const gemm::Args &args, int grid,
+                      cudaStream_t s)
+{
+    static bool configured = false;  // per process; attribute is per function
+    if (!configured) {
+        if (cudaFuncSetAttribute(gemm::grouped_gemm_kernel<kEpi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 gemm::SMEM_BYTES) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        configured = true;
+    }
+    gemm::grouped_gemm_kernel<kEpi><<<grid, gemm::NUM_THREADS, gemm::SMEM_BYTES, s>>>(a, b, args);
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int launch_grouped_gemm(int op, const moe_dims &d, int64_t R_cap, const int32_t *offsets, const moe_gemm_args &g,
+                        int *status, uint64_t budget, cudaStream_t s)
+{
+    gemm::Args a{};
+    a.offsets = offsets;
+    a.E = d.E;
+    a.R_cap = R_cap;
+    a.sa = g.sa;
+    a.sb = g.sb;
+    a.aux = g.aux;
+    a.out_q = g.out_q;
+    a.out_s = g.out_s;
+    a.out_bf16 = g.out_bf16;
+    a.out_f32 = g.out_f32;
+    a.status = status;
+    a.budget = budget;
+    CUtensorMap mA, mB;
+    const int64_t D = d.D, I = d.I, E = d.E;
+    bool ok = true;
+    switch (op) {
+    case MOE_GEMM_GATEUP_SILU:
+        a.N = (int)(2 * I); a.K = (int)D;
+        ok = make_map(&mA, g.a, D, R_cap, 128) && make_map(&mB, g.b, D, E * 2 * I, 256);
+        break;
+    case MOE_GEMM_DOWN:
+        a.N = (int)D; a.K = (int)I;
+        ok = make_map(&mA, g.a, I, R_cap, 128) && make_map(&mB, g.b, I, E * D, 256);
+        break;
+    case MOE_GEMM_DGRAD_DOWN_SILU:
+        a.N = (int)I; a.K = (int)D;
+        ok = make_map(&mA, g.a, D, R_cap, 128) && make_map(&mB, g.b, D, E * I, 256);
+        break;
+    case MOE_GEMM_DGRAD_GATEUP:
+        a.N = (int)D; a.K = (int)(2 * I);
+        ok = make_map(&mA, g.a, 2 * I, R_cap, 128) && make_map(&mB, g.b, 2 * I, E * D, 256);
+        break;
+    case MOE_GEMM_WGRAD_DOWN:
+        a.M = (int)D; a.N = (int)I;
+        ok = make_map(&mA, g.a, R_cap, D, 128) && make_map(&mB, g.b, R_cap, I, 256);
+        break;
+    case MOE_GEMM_WGRAD_GATEUP:
+        a.M = (int)(2 * I); a.N = (int)D;
+        ok = make_map(&mA, g.a, R_cap, 2 * I, 128) && make_map(&mB, g.b, R_cap, D, 256);
+        break;
+    default:
+        return MOE_ERR_INVALID_ARG;
+    }
+    if (!ok) return MOE_ERR_CUDA;
+    const int grid = sm_count();
+    switch (op) {
+    case MOE_GEMM_GATEUP_SILU: return launch_one<gemm::EPI_SILU>(mA, mB, a, grid, s);
+    case MOE_GEMM_DOWN:
+    case MOE_GEMM_DGRAD_GATEUP: return launch_one<gemm::EPI_BF16>(mA, mB, a, grid, s);
+    case MOE_GEMM_DGRAD_DOWN_SILU: return launch_one<gemm::EPI_DSILU>(mA, mB, a, grid, s);
+    default: return launch_one<gemm::EPI_WGRAD>(mA, mB, a, grid, s);
+    }
+}
+
+}  // namespace moe

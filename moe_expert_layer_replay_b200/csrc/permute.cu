@@ -1,0 +1,148 @@
+// a3: per-expert histogram, exclusive scan and stable permutation index.
+//
+// Dispatch groups each layer's routed token copies by expert ("RL at 1T
+// scale: prime-rl performance deep dive", §Wide Expert Parallelism and
+// §Parallelism/EP).  Routed entry i = t*k + j goes to row
+//     pos[i] = offsets[e] + #{ i' < i : idx[i'] = e },   e = idx[i],
+// with every expert's segment padded to a multiple of `align` rows.
+//
+// Three deterministic passes (no global atomics, so the result never depends
+// on scheduling):
+//   count: block b counts its chunk of entries per expert (shared atomics);
+//   scan:  per expert, an exclusive scan of the block counts (block bases),
+//          totals, then padded offsets;
+//   place: block b ranks its chunk in order; within a warp, peers with the
+//          same expert are found with match.any and ranked by lane order.
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int kChunk = 4096;  // entries per block
+constexpr int kPlaceWarps = 8;
+
+size_t permute_ws_bytes(int T, int k, int E)
+{
+    int64_t n = (int64_t)T * k;
+    int64_t nblk = (n + kChunk - 1) / kChunk;
+    if (nblk == 0) nblk = 1;
+    return (size_t)(2 * nblk * E) * sizeof(int32_t);
+}
+
+__global__ void __launch_bounds__(256) perm_count_kernel(const int32_t *__restrict__ idx, int64_t n,
+                                                         int E, int32_t *__restrict__ blkcnt)
+{
+    extern __shared__ int hist[];
+    for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+    __syncthreads();
+    int64_t base = (int64_t)blockIdx.x * kChunk;
+    for (int i = threadIdx.x; i < kChunk; i += blockDim.x) {
+        int64_t g = base + i;
+        if (g < n) {
+            int e = idx[g];
+            if (e >= 0 && e < E) atomicAdd(&hist[e], 1);
+        }
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) blkcnt[(int64_t)blockIdx.x * E + e] = hist[e];
+}
+
+__global__ void __launch_bounds__(256) perm_scan_kernel(const int32_t *__restrict__ blkcnt, int nblk,
+                                                        int E, int align,
+                                                        int32_t *__restrict__ blkbase,
+                                                        int32_t *__restrict__ counts,
+                                                        int32_t *__restrict__ offsets)
+{
+    __shared__ int padded[256];
+    int e = threadIdx.x;
+    if (e < E) {
+        int run = 0;
+        for (int b = 0; b < nblk; ++b) {
+            blkbase[(int64_t)b * E + e] = run;
+            run += blkcnt[(int64_t)b * E + e];
+        }
+        counts[e] = run;
+        padded[e] = (run + align - 1) / align * align;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int acc = 0;
+        offsets[0] = 0;
+        for (int i = 0; i < E; ++i) {
+            acc += padded[i];
+            offsets[i + 1] = acc;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(256) perm_place_kernel(const int32_t *__restrict__ idx, int64_t n,
+                                                         int E, const int32_t *__restrict__ blkbase,
+                                                         const int32_t *__restrict__ offsets,
+                                                         int32_t *__restrict__ pos,
+                                                         int32_t *__restrict__ src_idx, int *status)
+{
+    extern __shared__ int whist[];  // [kPlaceWarps][E]
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    for (int i = threadIdx.x; i < kPlaceWarps * E; i += blockDim.x) whist[i] = 0;
+    __syncthreads();
+    constexpr int sub = kChunk / kPlaceWarps;
+    const int64_t s0 = (int64_t)blockIdx.x * kChunk + (int64_t)wid * sub;
+    for (int i = lane; i < sub; i += 32) {
+        int64_t g = s0 + i;
+        if (g < n) {
+            int e = idx[g];
+            if (e >= 0 && e < E) atomicAdd(&whist[wid * E + e], 1);
+        }
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int run = offsets[e] + blkbase[(int64_t)blockIdx.x * E + e];
+        for (int w = 0; w < kPlaceWarps; ++w) {
+            int c = whist[w * E + e];
+            whist[w * E + e] = run;
+            run += c;
+        }
+    }
+    __syncthreads();
+    const unsigned lt = (1u << lane) - 1u;
+    for (int i0 = 0; i0 < sub; i0 += 32) {
+        int64_t g = s0 + i0 + lane;
+        bool in = g < n;
+        int e = in ? idx[g] : -1;
+        bool valid = in && e >= 0 && e < E;
+        unsigned peers = __match_any_sync(kFull, valid ? e : -1);
+        if (valid) {
+            int p = whist[wid * E + e] + __popc(peers & lt);
+            pos[g] = p;
+            src_idx[p] = (int32_t)g;
+        } else if (in) {
+            pos[g] = -1;
+            latch_status(status, MOE_ERR_BAD_ROUTING);
+        }
+        __syncwarp();
+        if (valid && (peers & lt) == 0) whist[wid * E + e] += __popc(peers);
+        __syncwarp();
+    }
+}
+
+int launch_permute_index(const int32_t *idx, int T, int k, int E, int align, int32_t *counts,
+                         int32_t *offsets, int32_t *pos, int32_t *src_idx, int64_t R_cap,
+                         void *ws, int *status, cudaStream_t s)
+{
+    int64_t n = (int64_t)T * k;
+    int nblk = (int)((n + kChunk - 1) / kChunk);
+    int32_t *blkcnt = (int32_t *)ws;
+    int32_t *blkbase = blkcnt + (int64_t)(nblk ? nblk : 1) * E;
+    if (cudaMemsetAsync(src_idx, 0xff, (size_t)R_cap * sizeof(int32_t), s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (nblk > 0) {
+        perm_count_kernel<<<nblk, 256, E * sizeof(int), s>>>(idx, n, E, blkcnt);
+    }
+    perm_scan_kernel<<<1, 256, 0, s>>>(blkcnt, nblk, E, align, blkbase, counts, offsets);
+    if (nblk > 0) {
+        perm_place_kernel<<<nblk, 32 * kPlaceWarps, kPlaceWarps * E * sizeof(int), s>>>(
+            idx, n, E, blkbase, offsets, pos, src_idx, status);
+    }
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // namespace moe

@@ -1,0 +1,63 @@
+"""Test helpers: host<->device marshalling and the parity tolerance.
+
+Tolerance for floating-point outputs (from the parity contract of the layer):
+relative Frobenius error <= 2e-3 and max-abs error <= 2e-2 * rms(reference).
+"""
+import numpy as np
+import torch
+
+REL_FRO = 2e-3
+MAX_ABS_RMS = 2e-2
+
+
+def dev(a, dtype=None):
+    """numpy -> cuda tensor (uint16 arrays become bf16 tensors)."""
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint16:
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()
+    t = torch.from_numpy(a).cuda()
+    return t if dtype is None else t.to(dtype)
+
+
+def host(t):
+    """cuda tensor -> numpy (bf16 -> uint16 bit patterns)."""
+    t = t.detach().contiguous()
+    if t.dtype == torch.bfloat16:
+        return t.cpu().view(torch.int16).numpy().view(np.uint16)
+    return t.cpu().numpy()
+
+
+def bf(a):
+    """bf16 bit patterns -> float64."""
+    return (np.asarray(a, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def close(got, ref, rel_fro=REL_FRO, max_abs_rms=MAX_ABS_RMS, what=""):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert got.shape == ref.shape, (what, got.shape, ref.shape)
+    assert np.all(np.isfinite(got)), what
+    nref = np.linalg.norm(ref)
+    err = np.linalg.norm(got - ref)
+    rms = np.sqrt(np.mean(ref ** 2)) if ref.size else 0.0
+    rel = err / nref if nref > 0 else err
+    mx = np.max(np.abs(got - ref)) if ref.size else 0.0
+    assert rel <= rel_fro, f"{what}: relative Frobenius error {rel:.3e} > {rel_fro}"
+    assert mx <= max_abs_rms * rms + 1e-30, f"{what}: max-abs error {mx:.3e} > {max_abs_rms} * rms {rms:.3e}"
+    return rel, mx
+
+
+def same_bits(got, ref, what=""):
+    got = np.ascontiguousarray(got)
+    ref = np.ascontiguousarray(ref)
+    assert got.shape == ref.shape, (what, got.shape, ref.shape)
+    if got.dtype == np.float32:
+        got, ref = got.view(np.int32), ref.view(np.int32)
+    bad = np.nonzero(got != ref)
+    assert len(bad[0]) == 0, f"{what}: {len(bad[0])} mismatches, first at {tuple(b[0] for b in bad)}: " \
+                             f"{got[tuple(b[0] for b in bad)]} vs {ref[tuple(b[0] for b in bad)]}"
+
+
+def rand_bf16(rng, shape, std=1.0):
+    from moe_expert_layer_replay_b200.inputs import to_bf16_bits
+    return to_bf16_bits(rng.standard_normal(shape).astype(np.float32) * np.float32(std))

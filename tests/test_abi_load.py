@@ -1,0 +1,41 @@
+"""The C-ABI library builds, loads without a GPU, and exports every entry
+point include/moe.h declares.  No compute call is made here."""
+import ctypes
+import os
+import re
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    from moe_expert_layer_replay_b200 import abi, build
+    build.build()
+    lib = ctypes.CDLL(abi.LIB_PATH)
+    names = _declared()
+    assert len(names) >= 14
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(abi.EXPORTS) == names
+
+
+def test_host_only_calls():
+    from moe_expert_layer_replay_b200 import abi
+    d = abi.dims(4096, 2048, 1024, 64, 6)
+    assert abi.rows_capacity(d) == (4096 * 6 + 64 * 127 + 127) // 128 * 128
+    assert abi.permute_workspace_size(d) > 0
+    assert abi.strerror(abi.BAD_ROUTING).startswith("routing")
+    # argument checks run before any device work
+    for bad in [abi.dims(16, 200, 128, 8, 2), abi.dims(16, 256, 128, 300, 2), abi.dims(16, 256, 128, 8, 9)]:
+        st = abi.lib().moe_route_topk(None, ctypes.byref(bad), None, None, None)
+        assert st in (abi.INVALID_ARG, abi.UNSUPPORTED)
+    g = abi.GemmArgs()
+    assert abi.lib().moe_grouped_gemm_fp8(0, ctypes.byref(abi.dims(16, 256, 100, 8, 2)), None,
+                                          ctypes.byref(g), None) == abi.UNSUPPORTED
+    assert abi.lib().moe_grouped_gemm_fp8(0, ctypes.byref(abi.dims(16, 256, 128, 8, 2)), None,
+                                          ctypes.byref(g), None) == abi.INVALID_ARG
