@@ -1,0 +1,346 @@
+"""Benchmark of the MoE expert layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload (default): the router-replay forward — T=4096 tokens, d_model=2048,
+expert FFN I=1024 (SiLU-gated), E=64 experts, top-6, routing replayed from a
+[L=4, 6, 4096] int32 payload (Zipf(1.1) expert popularity, Dirichlet(1)
+weights), bf16 N(0,1) activations, N(0,0.02) weights quantised once to
+128x128 FP8 blocks.  One step = the layer forward for each of the L=4
+replayed routings (replay -> permute + FP8 dispatch -> grouped GEMM gate/up +
+SiLU + h-quant -> grouped GEMM down -> combine), all with one set of expert
+weights.  value = L*T / step time (layer-tokens/s, i.e. the per-layer mean).
+
+N > 1 (torchrun, one rank per GPU): replicas — every rank runs its own batch
+(seed + rank) with the same weights; the layer has no cross-GPU exchange in
+data parallelism.  Timing is on the device, max over ranks.
+
+--impl reference times the CPU oracle (test infrastructure, fp64) on the host
+cores on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s; grouped FP8 GEMM TFLOP/s as % of dense FP8 peak"
+UNIT = "tokens/s"
+FP8_OVER_BF16 = 2.0  # nominal dense ratio (4.5 / 2.25 PFLOP/s)
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            pk = json.load(f)
+        return pk["hbm_gbs"], pk["bf16_tflops"], pk.get("bf16_tflops_sustained"), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def _workload_desc(wl):
+    return (f"{wl.name}: T={wl.T} D={wl.D} I={wl.I} E={wl.E} k={wl.k} L={wl.L} routing={wl.routing}"
+            + (f" zipf={wl.zipf}" if wl.zipf else ""))
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons during a region."""
+
+    def __init__(self, index: int, path: str):
+        self.path = path
+        self.p = None
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.f = open(path, "w")
+            self.p = subprocess.Popen(["nvidia-smi", f"--id={index}", f"--query-gpu={q}",
+                                       "--format=csv,noheader,nounits", "-lms", "200"],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return None
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except Exception:
+            self.p.kill()
+        self.f.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------
+# reference arm / CPU baseline: the oracle on host cores
+# --------------------------------------------------------------------------
+
+def oracle_sample_step(inp, wq, tokens: int, layer: int = 0):
+    """One bounded sample of the workload through the oracle: replay and
+    permute of all T tokens of layer `layer`, then the expert FFN and combine
+    of `tokens` evenly spaced tokens."""
+    import oracle
+    from oracle import layer as OL
+    wl = inp["workload"]
+    idx, w, st = oracle.route_replay(inp["payload"], layer, wl.E, w_in=inp["w_in"][layer])
+    sample = np.arange(tokens) * (wl.T // tokens)
+    return OL.forward_tokens(inp["x"], idx, w, wq, sample)["y"]
+
+
+def oracle_weights(inp):
+    from oracle import layer as OL
+    return (OL.quant_weights(inp["W_gate"]), OL.quant_weights(inp["W_up"]), OL.quant_weights(inp["W_down"]))
+
+
+def cpu_baseline(inp, tokens: int, reps: int = 1):
+    import oracle
+    wq = oracle_weights(inp)
+    t0 = time.perf_counter()
+    for r in range(reps):
+        oracle_sample_step(inp, wq, tokens, layer=r % inp["workload"].L)
+    dt = time.perf_counter() - t0
+    return {"value": reps * tokens / dt, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{tokens} tokens x {reps} layer pass(es) of the same workload through the fp64 oracle "
+                      f"(weights quantised once, outside the timing); {dt:.1f} s"}
+
+
+def run_reference(args, wl_name):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from moe_expert_layer_replay_b200.inputs import make_inputs
+    inp = make_inputs(wl_name, seed=args.seed)
+    wl = inp["workload"]
+    wq = oracle_weights(inp)
+    for _ in range(args.warmup):
+        oracle_sample_step(inp, wq, args.ref_tokens)
+    times = []
+    for s in range(args.steps):
+        t0 = time.perf_counter()
+        oracle_sample_step(inp, wq, args.ref_tokens, layer=s % wl.L)
+        times.append(time.perf_counter() - t0)
+    import oracle
+    tot = sum(times)
+    val = args.steps * args.ref_tokens / tot
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": _workload_desc(wl), "sample_tokens_per_step": args.ref_tokens},
+            "cpu_baseline": {"value": val, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+                             "sample": f"{args.ref_tokens} tokens of one replayed layer per step"},
+            "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------
+# our arm
+# --------------------------------------------------------------------------
+
+def run_ours(args, wl_name):
+    import torch
+    import torch.distributed as dist
+
+    from moe_expert_layer_replay_b200 import abi, layer
+    from moe_expert_layer_replay_b200.inputs import make_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local))
+    abi.lib()
+
+    inp = make_inputs(wl_name, seed=args.seed + rank)
+    wl = inp["workload"]
+    d = abi.dims(wl.T, wl.D, wl.I, wl.E, wl.k)
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16) if a.dtype == np.uint16 else
+                                     np.ascontiguousarray(a)).cuda()
+    bfd = lambda a: dev(a).view(torch.bfloat16)
+    W = layer.quantise_weights(d, bfd(inp["W_gate"]), bfd(inp["W_up"]), bfd(inp["W_down"]), train=False)
+    B = layer.Buffers(d, "cuda", train=False)
+    x = bfd(inp["x"])
+    payload = dev(inp["payload"])
+    w_in = dev(inp["w_in"])  # [L, T, k]
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    gemm1_events = []
+
+    def step(timed_gemm: bool):
+        for l in range(wl.L):
+            layer.route(B, payload=payload, layer=l, w_in=w_in[l])
+            # forward, with the gate/up GEMM bracketed by events when asked
+            abi.permute(B.idx, d, B.counts, B.offsets, B.pos, B.src, x, B.xq, B.xs, None, None, B.ws)
+            if timed_gemm:
+                e0, e1 = ev(), ev()
+                e0.record(stream)
+            abi.grouped_gemm_fp8(abi.GEMM_GATEUP_SILU, d, B.offsets, B.xq, B.xs, W.wgu_q, W.wgu_s,
+                                 out_q=B.hq, out_s=B.hs)
+            if timed_gemm:
+                e1.record(stream)
+                gemm1_events.append((e0, e1))
+            abi.grouped_gemm_fp8(abi.GEMM_DOWN, d, B.offsets, B.hq, B.hs, W.wd_q, W.wd_s, out_bf16=B.Y)
+            abi.combine(B.Y, B.w, B.pos, d, B.y)
+
+    launches_per_step = wl.L * (1 + 5 + 1 + 1 + 1)  # replay, permute (count/scan/place/quant/pad), 2 GEMMs, combine
+
+    for _ in range(max(3, args.warmup)):
+        step(False)
+    torch.cuda.synchronize()
+    st = abi.get_status()
+    if st != abi.OK:
+        raise RuntimeError(f"device status after warm-up: {abi.strerror(st)}")
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    clocks = Clocks(local, os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv")) \
+        if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else Clocks(local, f"/tmp/moe_clocks_{rank}.csv")
+    barrier()
+    step_ms = []
+    for _ in range(args.steps):
+        flush.fill_(1)  # L2 flush between timed steps, outside the events
+        e0, e1 = ev(), ev()
+        e0.record(stream)
+        step(True)
+        e1.record(stream)
+        step_ms.append((e0, e1))
+    barrier()
+    clk = clocks.stop()
+    step_ms = [a.elapsed_time(b) for a, b in step_ms]
+    g1_ms = [a.elapsed_time(b) for a, b in gemm1_events]
+    tot_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([tot_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        tot_ms = float(t.item())
+    ms_per_step = tot_ms / args.steps
+    value = world * wl.L * wl.T * args.steps / (tot_ms / 1e3)
+
+    # ---------------- end to end through the C ABI with host buffers
+    xh = torch.from_numpy(inp["x"].view(np.int16)).pin_memory()
+    ph = torch.from_numpy(inp["payload"]).pin_memory()
+    wh = torch.from_numpy(inp["w_in"]).pin_memory()
+    yh = torch.empty(wl.L, wl.T, wl.D, dtype=torch.int16).pin_memory()
+    xd = torch.empty_like(x)
+
+    def e2e_step():
+        xd.view(torch.int16).copy_(xh, non_blocking=True)
+        payload.copy_(ph, non_blocking=True)
+        w_in.copy_(wh, non_blocking=True)
+        for l in range(wl.L):
+            layer.route(B, payload=payload, layer=l, w_in=w_in[l])
+            layer.forward(B, xd, W)
+            yh[l].copy_(B.y.view(torch.int16), non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    barrier()
+    e0, e1 = ev(), ev()
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    barrier()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_val = world * wl.L * wl.T * args.steps / (e2e_ms / 1e3)
+    h2d = xh.numel() * 2 + ph.numel() * 4 + wh.numel() * 4
+    d2h = yh.numel() * 2
+
+    st = abi.get_status()
+    if st != abi.OK:
+        raise RuntimeError(f"device status after timing: {abi.strerror(st)}")
+
+    if rank == 0:
+        hbm, bf16_tf, bf16_sus, src = _peaks()
+        fp8_peak = bf16_tf * FP8_OVER_BF16
+        R = wl.T * wl.k
+        g1_flop = 2.0 * R * wl.D * (2 * wl.I)
+        g1_avg = statistics.mean(g1_ms)
+        achieved = g1_flop / (g1_avg / 1e3) / 1e12
+        gemm_tflops = wl.fwd_flop() * wl.L / (ms_per_step / 1e3) / 1e12  # whole-step view (lower bound)
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": max(3, args.warmup), "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "e4m3", "data": "synthetic",
+            "config": {"workload": _workload_desc(wl), "tokens_per_step_per_gpu": wl.L * wl.T,
+                       "l2": "flushed between timed steps (512 MiB write, outside the timed events)",
+                       "parallelism": "replicas" if world > 1 else "single GPU"},
+            "roofline": {"bound": "tensor", "kernel": "grouped_gemm gate/up + SiLU + h-quant",
+                         "achieved": achieved, "peak": fp8_peak, "unit": "TFLOP/s", "frac": achieved / fp8_peak,
+                         "traffic": None,
+                         "peak_note": f"fp8 dense = {FP8_OVER_BF16} x {src} bf16 burst {bf16_tf} TFLOP/s",
+                         "algorithmic": f"2*R*D*2I = {g1_flop:.4g} FLOP per launch (R = T*k routed rows)",
+                         "avg_launch_ms": g1_avg},
+            "gemm_tflops_step": gemm_tflops,
+            "gemm_frac_fp8_peak_step": gemm_tflops / fp8_peak,
+            "e2e": {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk,
+        }
+        if not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(inp, args.cpu_tokens)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="replay")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--cpu-tokens", type=int, default=1024)
+    ap.add_argument("--ref-tokens", type=int, default=128)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args, args.workload)
+    return run_ours(args, args.workload)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -110,7 +110,7 @@ def forward(x_bf16, idx, w, Wg_bf16, Wu_bf16, Wd_bf16, align: int = 128, quantis
     Returns a dict with every intermediate the GPU path also produces.
     """
     T, k = idx.shape
-    E = Wg_bf16.shape[0]
+    E = Wg_bf16.shape[0] if Wg_bf16 is not None else quantised_w[0][0].shape[0]
     counts, offsets, pos, src = permute(idx, E, align)
     R_pad = int(offsets[E])
     rows = np.arange(R_pad)
@@ -130,6 +130,36 @@ def forward(x_bf16, idx, w, Wg_bf16, Wu_bf16, Wd_bf16, align: int = 128, quantis
     return dict(counts=counts, offsets=offsets, pos=pos, src=src, Xp=Xp, xq=xq, xs=xs,
                 g=g, u=u, g_b=bf16_round(g), u_b=bf16_round(u), h=h, hq=hq, hs=hs,
                 Y=Y, y=y, expert=expert, Wq=quantised_w)
+
+
+def forward_tokens(x_bf16, idx, w, quantised_w, tokens, align: int = 128):
+    """Forward outputs of a sample of tokens, one token at a time.
+
+    Runs the permutation over all T tokens (it decides each routed row's
+    expert), then the expert FFN only for the rows the sampled tokens occupy:
+    for token t and slot j, row pos[t, j] holds x[t] quantised in 1x128
+    blocks (quantisation is row-local, so this equals that row of the full
+    dispatch).  Returns a dict with, per sampled token, its rows' h, hq, hs,
+    Y and the combined y.
+    """
+    T, k = idx.shape
+    Wg, Wu, Wd = quantised_w
+    E = Wg[0].shape[0]
+    counts, offsets, pos, src = permute(idx, E, align)
+    tokens = np.asarray(tokens, np.int64)
+    rows = pos[tokens].reshape(-1)                       # [n*k]
+    ok = rows >= 0
+    xr = np.repeat(x_bf16[tokens], k, axis=0)            # row (t, j) holds x[t]
+    xq, xs = quant_block(xr, 1, 128)
+    expert = np.where(ok, expert_of_rows(offsets, np.where(ok, rows, 0)), -1).astype(np.int32)
+    g, u = gateup_rows(xq, xs, expert, Wg, Wu)
+    h = swiglu_h(g, u)
+    hq, hs = quant_block(h, 1, 128)
+    Y = down_rows(hq, hs, expert, Wd)
+    n = len(tokens)
+    Yg = bf16_to_f64(Y).reshape(n, k, -1)
+    y = combine(Yg, w[tokens], ok.reshape(n, k))
+    return dict(rows=rows.reshape(n, k), h=h, hq=hq, hs=hs, Y=Y, y=y, offsets=offsets, pos=pos)
 
 
 # --------------------------------------------------------------------------

@@ -300,12 +300,24 @@ typedef struct {
     int64_t nr, nc;
 } orc_wmat;
 
+/* Values of all 256 codes, filled once from orc_e4m3_to_double (a lookup
+ * instead of a decode per element; identical values). */
+static double e4m3_value[256];
+static int e4m3_value_ready = 0;
+
+static void e4m3_table_init(void)
+{
+    if (e4m3_value_ready) return;
+    for (int c = 0; c < 256; ++c) e4m3_value[c] = orc_e4m3_to_double((uint8_t)c);
+    e4m3_value_ready = 1;
+}
+
 static double wmat_get(const orc_wmat *W, int64_t e, int64_t r, int64_t c)
 {
     if (W->f) return W->f[(e * W->nr + r) * W->nc + c];
     int64_t gbr = (W->nr + 127) / 128, gbc = (W->nc + 127) / 128;
     double sc = W->s[(e * gbr + r / 128) * gbc + c / 128];
-    return orc_e4m3_to_double(W->q[(e * W->nr + r) * W->nc + c]) * sc;
+    return e4m3_value[W->q[(e * W->nr + r) * W->nc + c]] * sc;
 }
 
 /* out[i][n] = sum_c A[i][c] * W[e_i][n][c]           (trans = 0; W is [N][K])
@@ -318,6 +330,7 @@ void orc_rowdot(const double *A, int64_t n_rows, const int32_t *expert, int E,
 {
     orc_wmat W = {Wq, Ws, Wf, w_nr, w_nc};
     int64_t K = trans ? w_nr : w_nc, N = trans ? w_nc : w_nr;
+    e4m3_table_init();
     for (int64_t i = 0; i < n_rows * N; ++i) out[i] = 0.0;
     for (int e = 0; e < E; ++e) {
         int64_t cnt = 0;

@@ -8,6 +8,14 @@ import torch
 
 REL_FRO = 2e-3
 MAX_ABS_RMS = 2e-2
+# End-to-end comparisons (oracle run from the raw inputs alone) of outputs that
+# lie downstream of an FP8 re-quantisation of a float intermediate (h, d[g|u]):
+# the two sides compute that intermediate in different precision (fp32 vs fp64
+# accumulation), so an element can land on the neighbouring e4m3 code (a
+# relative step of up to 2^-3 of that element).  The relative Frobenius bound
+# stays; the max-abs bound is 5e-2 * rms there.  Per-step comparisons, on
+# identical inputs, use the contract bounds above.
+MAX_ABS_RMS_E2E = 5e-2
 
 
 def dev(a, dtype=None):

@@ -10,7 +10,7 @@ import numpy as np
 import pytest
 import torch
 
-from _util import bf, close, dev, host, rand_bf16, same_bits
+from _util import MAX_ABS_RMS_E2E, bf, close, dev, host, rand_bf16, same_bits
 
 pytestmark = pytest.mark.gpu
 
@@ -77,7 +77,7 @@ def test_layer_parity(A, orc, case):
     same_bits(host(B.pos), fw["pos"], "pos")
     same_bits(host(B.xq)[:Rp], fw["xq"], "xq")
     same_bits(host(B.xs)[:, :Rp].T, fw["xs"], "xs")
-    close(bf(host(B.y)), bf(fw["y"]), what="y end to end")
+    close(bf(host(B.y)), bf(fw["y"]), max_abs_rms=MAX_ABS_RMS_E2E, what="y end to end")
 
     # ---- GEMM1 step on the same (bit-exact) operands
     hg = host(h_gpu)[:Rp]
@@ -99,18 +99,9 @@ def test_layer_parity(A, orc, case):
 
     if not train:
         return
-    # ---- backward, end to end
     bw = OL.backward(fw, x, dy, idx, w, z=z)
-    close(bf(host(B.dx)), bf(bw["dx"]), what="dx end to end")
-    close(host(B.d_w), bw["d_w"], what="d_w")
-    close(host(B.d_logits), bw["dz"], what="d_logits")
     dWd = host(B.dWd)
     dWgu = host(B.dWgu)
-    dWg = np.concatenate([dWgu[:, 256 * b:256 * b + 128] for b in range(I // 128)], axis=1)
-    dWu = np.concatenate([dWgu[:, 256 * b + 128:256 * b + 256] for b in range(I // 128)], axis=1)
-    close(dWd, bw["dWd"], what="dW_down end to end")
-    close(dWg, bw["dWg"], what="dW_gate end to end")
-    close(dWu, bw["dWu"], what="dW_up end to end")
 
     # ---- backward steps on the GPU's own upstream operands
     expert = fw["expert"]
@@ -156,6 +147,17 @@ def test_layer_parity(A, orc, case):
         close(dWd[e], OL.wgrad_expert(dYqT, dYsT, hqT, hsT, r0, r1), what=f"dW_down[{e}]")
         close(dWgu[e], OL.wgrad_expert(host(B.dGUqT)[:, :Rp].T.copy(), host(B.dGUsT)[:Rp // 128],
                                        xqT, xsT, r0, r1), what=f"dW_gate_up[{e}]")
+
+    # ---- backward, end to end from the raw inputs
+    close(host(B.d_w), bw["d_w"], what="d_w")          # upstream of any re-quantisation
+    close(host(B.d_logits), bw["dz"], what="d_logits")
+    e2e = dict(max_abs_rms=MAX_ABS_RMS_E2E)
+    close(bf(host(B.dx)), bf(bw["dx"]), what="dx end to end", **e2e)
+    dWg = np.concatenate([dWgu[:, 256 * b:256 * b + 128] for b in range(I // 128)], axis=1)
+    dWu = np.concatenate([dWgu[:, 256 * b + 128:256 * b + 256] for b in range(I // 128)], axis=1)
+    close(dWd, bw["dWd"], what="dW_down end to end", **e2e)
+    close(dWg, bw["dWg"], what="dW_gate end to end", **e2e)
+    close(dWu, bw["dWu"], what="dW_up end to end", **e2e)
 
 
 def test_layer_deterministic(A):
