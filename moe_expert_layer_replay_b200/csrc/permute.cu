@@ -17,7 +17,7 @@
 
 namespace moe {
 
-constexpr int kChunk = 4096;  // entries per block
+constexpr int kChunk = 1024;  // entries per block
 constexpr int kPlaceWarps = 8;
 
 size_t permute_ws_bytes(int T, int k, int E)

@@ -57,7 +57,7 @@ def test_full_size_forward_sampled(A, orc, name, n_sample):
     same_bits(host(B.pos), op, "pos")
     same_bits(host(B.src), osrc, "src_idx")
     if name == "prefill":
-        assert np.sum(oc == 0) == 4 and oc.max() > 4 * oc.mean()   # skewed, with empty experts
+        assert np.sum(oc == 0) == 4 and oc.max() > 3 * oc.mean()   # skewed, with empty experts
 
     rng = np.random.default_rng(1)
     sample = np.sort(rng.choice(wl.T, n_sample, replace=False))
