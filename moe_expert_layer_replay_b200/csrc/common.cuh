@@ -57,24 +57,104 @@ __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi)
 // Scale of a block: fp32(amax / 448), IEEE division.
 __device__ __forceinline__ float block_scale(float amax) { return __fdiv_rn(amax, 448.0f); }
 
-// Four codes of fp32(v / s), s != 0.
-__device__ __forceinline__ uint32_t quant4(const float *v, float s)
+// The e4m3 code of the correctly rounded quotient q = RN_fp32(x / s),
+// without a divide per element.
+//
+// With r = RN(1/s), q' = RN(x * r) is within 2^-23 relative of x/s, so within
+// 2.5 fp32 ulps of q.  e4m3 (3 mantissa bits) rounds q and q' to different
+// codes only if an e4m3 rounding midpoint M lies between them.  In e4m3's
+// normal range a midpoint is an fp32 value whose 20 low mantissa bits are
+// 0x80000; q' is "near" when those bits are within 4 of it.  Below 2^-6
+// (e4m3's subnormal grid, step 2^-9) every element is treated as near.
+//
+// A near element is decided exactly against the midpoint M of its e4m3 cell:
+// q > M iff x/s > M + u/2, q < M iff x/s < M - u/2, else q == M (u = fp32 ulp
+// of M; M has 4 significant bits, so ties at M +- u/2 round to M).  The sign
+// of x - (M +- u/2) * s is exact in fp64: the product has 49 significant bits.
+// The element then converts through M (tie: even code) or its fp32 neighbour
+// on the decided side, which e4m3 rounds like q.  No midpoint is ever
+// decided by an approximation.
+__device__ __forceinline__ float near_midpoint_exact(float x, float s, float qp)
 {
-    return e4m3x2(__fdiv_rn(v[0], s), __fdiv_rn(v[1], s)) |
-           (e4m3x2(__fdiv_rn(v[2], s), __fdiv_rn(v[3], s)) << 16);
+    const float aq = fabsf(qp);
+    const uint32_t b = __float_as_uint(aq);
+    const float M = (b < 0x3c800000u) ? (floorf(aq * 512.0f) + 0.5f) * (1.0f / 512.0f)
+                                      : __uint_as_float((b & 0xfff00000u) | 0x00080000u);
+    const double half_ulp = (double)__uint_as_float(__float_as_uint(M) & 0x7f800000u) * 0x1p-24;
+    const double xd = (double)fabsf(x), sd = (double)s;
+    float v;
+    if (xd - ((double)M + half_ulp) * sd > 0.0) v = __uint_as_float(__float_as_uint(M) + 1u);
+    else if (xd - ((double)M - half_ulp) * sd < 0.0) v = __uint_as_float(__float_as_uint(M) - 1u);
+    else v = M;
+    return copysignf(v, x);
+}
+
+// IEEE division for a whole group; only for scales whose reciprocal is not
+// finite (amax below about 1.5e-36), kept out of line.
+template <int n>
+struct Floats {
+    float v[n];
+};
+
+template <int n>
+__device__ __noinline__ Floats<n> quotients_exact(Floats<n> x, float s)
+{
+    Floats<n> q;
+#pragma unroll
+    for (int i = 0; i < n; ++i) q.v[i] = __fdiv_rn(x.v[i], s);
+    return q;
+}
+
+// Values whose e4m3 conversion equals that of fp32(v[i] / s), s != 0.
+template <int n>
+__device__ __forceinline__ void quotients(const float *v, float s, float *q)
+{
+    const float r = __frcp_rn(s);
+    if (!(r <= 3.0e38f)) {
+        Floats<n> x;
+#pragma unroll
+        for (int i = 0; i < n; ++i) x.v[i] = v[i];
+        const Floats<n> e = quotients_exact<n>(x, s);
+#pragma unroll
+        for (int i = 0; i < n; ++i) q[i] = e.v[i];
+        return;
+    }
+#pragma unroll
+    for (int i = 0; i < n; ++i) {
+        q[i] = __fmul_rn(v[i], r);
+        const uint32_t b = __float_as_uint(q[i]) & 0x7fffffffu;
+        const int low = (int)(b & 0xfffffu) - 0x80000;
+        if ((b < 0x3c800000u && b != 0u) || (low >= -4 && low <= 4)) q[i] = near_midpoint_exact(v[i], s, q[i]);
+    }
 }
 
 // Sixteen codes; a zero scale gives zero codes.
 __device__ __forceinline__ uint4 quant16(const float *v, float s)
 {
     if (s == 0.0f) return make_uint4(0, 0, 0, 0);
-    return make_uint4(quant4(v, s), quant4(v + 4, s), quant4(v + 8, s), quant4(v + 12, s));
+    float q[16];
+    quotients<16>(v, s, q);
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) w[i] = e4m3x2(q[4 * i], q[4 * i + 1]) | (e4m3x2(q[4 * i + 2], q[4 * i + 3]) << 16);
+    return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
 __device__ __forceinline__ uint2 quant8(const float *v, float s)
 {
     if (s == 0.0f) return make_uint2(0, 0);
-    return make_uint2(quant4(v, s), quant4(v + 4, s));
+    float q[8];
+    quotients<8>(v, s, q);
+    return make_uint2(e4m3x2(q[0], q[1]) | (e4m3x2(q[2], q[3]) << 16),
+                      e4m3x2(q[4], q[5]) | (e4m3x2(q[6], q[7]) << 16));
+}
+
+// sigmoid(g) for the SiLU gate, fast intrinsics (h and its gradient are
+// compared within a tolerance, not bit for bit).  exp(80) < 2^126 keeps the
+// fast division in range; below g = -80 the sigmoid is 0 in fp32 anyway.
+__device__ __forceinline__ float sigmoid_fast(float g)
+{
+    return __fdividef(1.0f, 1.0f + __expf(-fmaxf(g, -80.0f)));
 }
 
 __device__ __forceinline__ float absmax8(const float *v, float m)

@@ -48,15 +48,21 @@ constexpr int EPI_WARP0 = 4;
 constexpr int EPI_THREADS = 256;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint64_t DRAIN_BUDGET = 1ull << 28;
-// smem: ring | barriers (full[4], empty[4], tfull[2], tempty[2], drain, epi) |
-// tmem slot | abort flag | offsets[257] | amax exchange [2][2][128] | wgrad col scales [2][256]
+constexpr int PF = 3;  // scale prefetch depth (K blocks)
+// smem: operand ring | barriers (full[4], empty[4], tfull[2], tempty[2], drain, epi) |
+// tmem slot | abort flag | offsets[257] | amax exchange [2][2][128] |
+// scale ring [PF][3][256] fp32 (per epilogue thread: row scale, weight/column
+// scale, second weight scale) | bf16 output staging [8 warps][32 rows][80 B]
 constexpr int OFF_BAR = STAGES * STAGE_BYTES;
 constexpr int OFF_TMEM_SLOT = OFF_BAR + 16 * 8;
 constexpr int OFF_ABORT = OFF_TMEM_SLOT + 4;
 constexpr int OFF_OFFSETS = OFF_BAR + 256;
 constexpr int OFF_AMAX = OFF_OFFSETS + 1040;
-constexpr int OFF_COLSCALE = OFF_AMAX + 2 * 2 * 128 * 4;
-constexpr int SMEM_BYTES = OFF_COLSCALE + 2 * 256 * 4 + 1024;  // + alignment slack
+constexpr int OFF_RING = OFF_AMAX + 2 * 2 * 128 * 4;
+constexpr int STAGE_ROW = 80;  // 64 B of bf16 + 16 B pad: conflict-free 16-byte rows
+constexpr int OFF_STAGE = OFF_RING + PF * 3 * 256 * 4;
+constexpr int SMEM_BYTES = OFF_STAGE + 8 * 32 * STAGE_ROW + 1024;  // + alignment slack
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
 enum Epi { EPI_SILU = 0, EPI_BF16 = 1, EPI_DSILU = 2, EPI_WGRAD = 3 };
 
@@ -120,15 +126,26 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, uint
 {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
-    while (true) {
+    for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (*abort_flag) return false;
-        if ((uint64_t)(clock64() - t0) > budget) {
-            *abort_flag = 1;
-            latch_status(status, MOE_ERR_TIMEOUT);
-            return false;
+        if ((it & 31u) == 0) {  // the budget and the abort flag are checked every 32 polls
+            if (*abort_flag) return false;
+            if ((uint64_t)(clock64() - t0) > budget) {
+                *abort_flag = 1;
+                latch_status(status, MOE_ERR_TIMEOUT);
+                return false;
+            }
         }
     }
+}
+
+// Warp-wide wait: lane 0 polls, the other lanes wait for its verdict.
+__device__ __forceinline__ bool warp_wait_bounded(uint32_t bar, uint32_t parity, uint64_t budget,
+                                                  volatile int *abort_flag, int *status)
+{
+    bool ok = true;
+    if ((threadIdx.x & 31) == 0) ok = wait_bounded(bar, parity, budget, abort_flag, status);
+    return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
 // Drain wait: ignores the abort flag (used on the way out).
@@ -147,6 +164,23 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
         " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
         : "memory");
+}
+
+__device__ __forceinline__ void cp_async4(void *dst, const void *src)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int n>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(n) : "memory"); }
+
+// a = fma(p, s, a) on two fp32 lanes at once (packed f32x2)
+__device__ __forceinline__ void ffma2(float &a0, float &a1, float p0, float p1, float s0, float s1)
+{
+    asm("{\n\t.reg .b64 a, p, q;\n\tmov.b64 a, {%0, %1};\n\tmov.b64 p, {%2, %3};\n\t"
+        "mov.b64 q, {%4, %5};\n\tfma.rn.f32x2 a, p, q, a;\n\tmov.b64 {%0, %1}, a;\n\t}"
+        : "+f"(a0), "+f"(a1)
+        : "f"(p0), "f"(p1), "f"(s0), "f"(s1));
 }
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -269,7 +303,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_TMEM_SLOT);
     int *offs_s = reinterpret_cast<int *>(smem + OFF_OFFSETS);
     float *amax_s = reinterpret_cast<float *>(smem + OFF_AMAX);       // [2][2][128]
-    float *colscale_s = reinterpret_cast<float *>(smem + OFF_COLSCALE);  // [2][256]
+    float *ring = reinterpret_cast<float *>(smem + OFF_RING);          // [PF][3][256]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -411,69 +445,103 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             float acc[128];
 #pragma unroll
             for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
-            // scale fetch for K block kb
-            auto fetch = [&](int kb, float &sa, float &s0, float &s1, float &cs) {
-                if (kWgrad) {
-                    sa = p.sa[(int64_t)kb * p.M + x.m0 + row];
-                    const int c = x.n0 + et;
-                    cs = (c < p.N) ? p.sb[(int64_t)kb * p.N + c] : 0.0f;
-                    s0 = s1 = 0.0f;
+            // Scales of K block kb.  Rows mode: plain loads two K blocks ahead
+            // into registers (row scale, weight-block scale(s)).  Wgrad: the
+            // column scales are shared by the warps, so they go through a
+            // cp.async ring in shared memory (slot kb % PF) read after a sync.
+            auto load_rows = [&](int kb, float &a, float &b0, float &b1) {
+                a = p.sa[(int64_t)kb * p.R_cap + x.m0 + row];
+                const int64_t sbrow = (int64_t)x.e * NB + 2 * x.nt;
+                if (kEpi == EPI_SILU) {
+                    b0 = p.sb[sbrow * KB + kb];        // gate block
+                    b1 = p.sb[(sbrow + 1) * KB + kb];  // up block
                 } else {
-                    sa = p.sa[(int64_t)kb * p.R_cap + x.m0 + row];
-                    const int64_t sbrow = (int64_t)x.e * NB + 2 * x.nt;
-                    if (kEpi == EPI_SILU) {
-                        s0 = p.sb[sbrow * KB + kb];        // gate block
-                        s1 = p.sb[(sbrow + 1) * KB + kb];  // up block
-                    } else {
-                        const int64_t nb = sbrow + h;
-                        s0 = s1 = (2 * x.nt + h < NB) ? p.sb[nb * KB + kb] : 0.0f;
-                    }
-                    cs = 0.0f;
+                    b0 = (2 * x.nt + h < NB) ? p.sb[(sbrow + h) * KB + kb] : 0.0f;
+                    b1 = b0;
                 }
             };
-            float n_sa, n_s0, n_s1, n_cs;
-            fetch(x.kb0, n_sa, n_s0, n_s1, n_cs);
+            auto issue_wgrad = [&](int kb) {
+                float *d = ring + (kb % PF) * 768;
+                cp_async4(d + et, p.sa + (int64_t)kb * p.M + x.m0 + row);
+                const int c = x.n0 + et;
+                if (c < p.N) cp_async4(d + 256 + et, p.sb + (int64_t)kb * p.N + c);
+            };
+            float c_a = 0.f, c_b0 = 0.f, c_b1 = 0.f, n_a = 0.f, n_b0 = 0.f, n_b1 = 0.f;
+            if (kWgrad) {
+                if (!epi_sync()) break;  // the previous tile's column scales are read
+#pragma unroll
+                for (int j = 0; j < PF - 1; ++j) {
+                    if (x.kb0 + j < x.kb1) issue_wgrad(x.kb0 + j);
+                    cp_async_commit();
+                }
+            } else {
+                load_rows(x.kb0, c_a, c_b0, c_b1);
+                if (x.kb0 + 1 < x.kb1) load_rows(x.kb0 + 1, n_a, n_b0, n_b1);
+            }
             for (int kb = x.kb0; kb < x.kb1; ++kb) {
-                const float sa = n_sa, s0 = n_s0, s1 = n_s1, cs = n_cs;
-                if (kb + 1 < x.kb1) fetch(kb + 1, n_sa, n_s0, n_s1, n_cs);
-                float *cscale = colscale_s + (kb & 1) * 256;
+                const float *d = ring + (kb % PF) * 768;
+                float sa, s0, s1;
                 if (kWgrad) {
-                    cscale[et] = cs;
-                    if (!epi_sync()) {
+                    cp_async_wait<PF - 2>();
+                    if (!epi_sync()) {  // everyone's column scales of kb are in
                         ok = false;
                         break;
                     }
+                    if (kb + PF - 1 < x.kb1) issue_wgrad(kb + PF - 1);
+                    cp_async_commit();
+                    sa = d[et];
+                    s0 = s1 = 0.0f;
+                } else {
+                    sa = c_a;
+                    s0 = c_a * c_b0;
+                    s1 = c_a * c_b1;
+                    c_a = n_a, c_b0 = n_b0, c_b1 = n_b1;
+                    if (kb + 2 < x.kb1) load_rows(kb + 2, n_a, n_b0, n_b1);
                 }
-                if (!wait_bounded(bar_tfull + 8 * buf, bphase, p.budget, abort_flag, p.status)) {
+                if (!warp_wait_bounded(bar_tfull + 8 * buf, bphase, p.budget, abort_flag, p.status)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 const uint32_t cbase = lane_addr + (uint32_t)(buf * BN);
+                auto col_of = [&](int c) -> uint32_t {
+                    if (kEpi == EPI_SILU) return (c < 2) ? (64 * h + 32 * c) : (128 + 64 * h + 32 * (c - 2));
+                    return 128 * h + 32 * c;
+                };
+                // TMEM reads pipelined one chunk ahead of the FMAs; the buffer
+                // goes back to the MMA as soon as the last read has landed
+                uint32_t ra[32], rb[32];
+                MOE_TMEM_LD32(cbase + col_of(0), ra);
+                tmem_wait_ld();
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    uint32_t col;
-                    if (kEpi == EPI_SILU) col = (c < 2) ? (64 * h + 32 * c) : (128 + 64 * h + 32 * (c - 2));
-                    else col = 128 * h + 32 * c;
-                    uint32_t r[32];
-                    MOE_TMEM_LD32(cbase + col, r);
-                    tmem_wait_ld();
+                    uint32_t *cur = (c & 1) ? rb : ra;
+                    uint32_t *nxt = (c & 1) ? ra : rb;
+                    if (c + 1 < 4) MOE_TMEM_LD32(cbase + col_of(c + 1), nxt);
                     if (kWgrad) {
+                        const float *cs = d + 256 + 128 * h + 32 * c;
 #pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            acc[32 * c + i] = fmaf(__uint_as_float(r[i]), sa * cscale[col + i], acc[32 * c + i]);
+                        for (int i = 0; i < 32; i += 2)
+                            ffma2(acc[32 * c + i], acc[32 * c + i + 1], __uint_as_float(cur[i]),
+                                  __uint_as_float(cur[i + 1]), sa * cs[i], sa * cs[i + 1]);
                     } else {
-                        const float sc = sa * ((kEpi == EPI_SILU && c >= 2) ? s1 : s0);
+                        const float sc = (kEpi == EPI_SILU && c >= 2) ? s1 : s0;
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) acc[32 * c + i] = fmaf(__uint_as_float(r[i]), sc, acc[32 * c + i]);
+                        for (int i = 0; i < 32; i += 2)
+                            ffma2(acc[32 * c + i], acc[32 * c + i + 1], __uint_as_float(cur[i]),
+                                  __uint_as_float(cur[i + 1]), sc, sc);
+                    }
+                    if (c + 1 < 4) tmem_wait_ld();
+                    if (c == 2) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bar_tempty + 8 * buf);
                     }
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar_tempty + 8 * buf);
                 buf ^= 1;
                 if (buf == 0) bphase ^= 1;
             }
+            cp_async_wait<0>();
             if (!ok) break;
             const int64_t r = (int64_t)x.m0 + row;
             // ------------------------------------------- fused outputs ----
@@ -492,7 +560,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 #pragma unroll
                     for (int i = i0; i < i0 + 8; ++i) {
                         const float g = acc[i], u = acc[64 + i];
-                        const float sg = g / (1.0f + expf(-g));
+                        const float sg = g * sigmoid_fast(g);
                         const float hv = __uint_as_float(bf16_bits_rn(sg * u) << 16);
                         acc[i] = hv;
                         amax = fmaxf(amax, fabsf(hv));
@@ -513,11 +581,26 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     for (int i0 = 0; i0 < 64; i0 += 8) *reinterpret_cast<uint4 *>(hb + i0) = pack8(&acc[i0]);
                 }
             } else if (kEpi == EPI_BF16) {
+                // through a per-warp smem tile, so that each store instruction
+                // writes 8 rows x 64 contiguous bytes instead of 32 scattered 16 B
                 const int64_t c0 = (int64_t)x.n0 + 128 * h;
                 if (c0 < p.N) {
-                    uint16_t *o = p.out_bf16 + r * p.N + c0;
+                    uint8_t *stg = smem + OFF_STAGE + ew * 32 * STAGE_ROW;
+                    const int64_t rbase = (int64_t)x.m0 + 32 * q;
 #pragma unroll
-                    for (int i0 = 0; i0 < 128; i0 += 8) *reinterpret_cast<uint4 *>(o + i0) = pack8(&acc[i0]);
+                    for (int ch = 0; ch < 4; ++ch) {
+                        uint4 *w = reinterpret_cast<uint4 *>(stg + lane * STAGE_ROW);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) w[j] = pack8(&acc[32 * ch + 8 * j]);
+                        __syncwarp();
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int rr = (lane & 7) + 8 * i, pc = lane >> 3;
+                            const uint4 v = *reinterpret_cast<const uint4 *>(stg + rr * STAGE_ROW + pc * 16);
+                            *reinterpret_cast<uint4 *>(p.out_bf16 + (rbase + rr) * p.N + c0 + 32 * ch + 8 * pc) = v;
+                        }
+                        __syncwarp();
+                    }
                 }
             } else if (kEpi == EPI_DSILU) {
                 // acc = dH of I-block nb = 2nt + h; gate/up columns of that block
@@ -537,7 +620,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
                             const float dh = acc[i0 + i];
-                            const float sg = 1.0f / (1.0f + expf(-g[i]));
+                            const float sg = sigmoid_fast(g[i]);
                             const float dgv = dh * u[i] * sg * (1.0f + g[i] * (1.0f - sg));
                             const float duv = dh * g[i] * sg;
                             const uint32_t bg = bf16_bits_rn(dgv), bu = bf16_bits_rn(duv);
@@ -584,6 +667,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 }
             }
         }
+        cp_async_wait<0>();  // no copy into shared memory outlives the CTA
     }
     tc_fence_before();
     __syncthreads();

@@ -70,11 +70,11 @@ def test_full_size_forward_sampled(A, orc, name, n_sample):
     same_bits(xq, oq, "dispatched codes (sample)")
     same_bits(xs, os_, "dispatched scales (sample)")
     hg = host(h[rows])
-    close(bf(hg), bf(ref["h"]), what="h (sample)")
+    close(bf(hg), bf(ref["h"]), bf16=True, what="h (sample)")
     hq_ref, hs_ref = orc.quant_block(hg, 1, 128)
     same_bits(host(B.hq[rows]), hq_ref, "hq = quant(h) (sample)")
     same_bits(host(B.hs[:, rows]).T, hs_ref, "hs = quant(h) (sample)")
     expert = OL.expert_of_rows(oo, rows)
     Y_ref = OL.down_rows(host(B.hq[rows]), host(B.hs[:, rows]).T.copy(), expert, wq[2])
-    close(bf(host(B.Y[rows])), bf(Y_ref), what="Y from the GPU's hq (sample)")
-    close(bf(host(B.y[sample])), bf(ref["y"]), max_abs_rms=MAX_ABS_RMS_E2E, what="y end to end (sample)")
+    close(bf(host(B.Y[rows])), bf(Y_ref), bf16=True, what="Y from the GPU's hq (sample)")
+    close(bf(host(B.y[sample])), bf(ref["y"]), bf16=True, max_abs_rms=MAX_ABS_RMS_E2E, what="y end to end (sample)")

@@ -224,11 +224,11 @@ def test_combine_and_unpermute(A, orc):
     y = torch.empty(T, D, dtype=torch.bfloat16, device="cuda")
     A.combine(dev(Y), dev(w), dev(op), d, y)
     ref = combine(bf(Y)[op], w, op >= 0)
-    close(bf(host(y)), bf(ref), what="combine")
+    close(bf(host(y)), bf(ref), bf16=True, what="combine")
     dx = torch.empty(T, D, dtype=torch.bfloat16, device="cuda")
     A.unpermute_reduce(dev(Y), dev(op), d, dx)
     ref = unpermute_reduce(bf(Y), op)
-    close(bf(host(dx)), bf(ref), what="unpermute")
+    close(bf(host(dx)), bf(ref), bf16=True, what="unpermute")
 
 
 def test_combine_bwd(A, orc):
@@ -256,3 +256,45 @@ def test_combine_bwd(A, orc):
     ref_dw, ref_dz = router_grads(dy, bf(Y)[op], w, z, idx)
     close(host(d_w), ref_dw, what="d_w")
     close(host(dz), ref_dz, what="d_logits")
+
+
+@pytest.mark.parametrize("blk", [(1, 128), (128, 1), (128, 128)])
+def test_quant_exhaustive_bf16(A, orc, blk):
+    """Every finite bf16 value, in blocks whose amax (hence scale) varies from
+    subnormal to large, quantises bit-exactly like the oracle's IEEE
+    definition (scale = fp32(amax/448), code = e4m3(fp32(x/scale)))."""
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    finite = (bits & 0x7F80) != 0x7F80
+    vals = bits[finite]
+    rng = np.random.default_rng(7)
+    rng.shuffle(vals)
+    n = (len(vals) + 16383) // 16384 * 16384
+    x = np.zeros(n, np.uint16)
+    x[:len(vals)] = vals
+    x = x.reshape(-1, 128)  # 512 rows x 128
+    # vary the block maxima: some blocks get a planted amax from subnormal to 1e30
+    planted = orc.bf16_round(np.logspace(-40, 30, x.shape[0]) * rng.choice([-1, 1], x.shape[0]))
+    x[np.arange(x.shape[0]), rng.integers(0, 128, x.shape[0])] = planted
+    br, bc = blk
+    rows, cols = x.shape
+    if br == 1:
+        q = torch.empty(rows, cols, dtype=torch.uint8, device="cuda")
+        s = torch.empty(cols // 128, rows, dtype=torch.float32, device="cuda")
+        A.quant_fp8_block(dev(x), rows, cols, cols, 1, 128, q, s)
+        oq, os_ = orc.quant_block(x, 1, 128)
+        same_bits(host(q), oq, "codes")
+        same_bits(host(s).T, os_, "scales")
+    elif bc == 1:
+        q = torch.empty(cols, rows, dtype=torch.uint8, device="cuda")
+        s = torch.empty(rows // 128, cols, dtype=torch.float32, device="cuda")
+        A.quant_fp8_block(dev(x), rows, cols, cols, 128, 1, q, s)
+        oq, os_ = orc.quant_block(x, 128, 1)
+        same_bits(host(q).T, oq, "codes")
+        same_bits(host(s), os_, "scales")
+    else:
+        q = torch.empty(rows, cols, dtype=torch.uint8, device="cuda")
+        s = torch.empty(rows // 128, 1, dtype=torch.float32, device="cuda")
+        A.quant_fp8_block(dev(x), rows, cols, cols, 128, 128, q, s)
+        oq, os_ = orc.quant_block(x, 128, 128)
+        same_bits(host(q), oq, "codes")
+        same_bits(host(s), os_, "scales")

@@ -77,11 +77,11 @@ def test_layer_parity(A, orc, case):
     same_bits(host(B.pos), fw["pos"], "pos")
     same_bits(host(B.xq)[:Rp], fw["xq"], "xq")
     same_bits(host(B.xs)[:, :Rp].T, fw["xs"], "xs")
-    close(bf(host(B.y)), bf(fw["y"]), max_abs_rms=MAX_ABS_RMS_E2E, what="y end to end")
+    close(bf(host(B.y)), bf(fw["y"]), bf16=True, max_abs_rms=MAX_ABS_RMS_E2E, what="y end to end")
 
     # ---- GEMM1 step on the same (bit-exact) operands
     hg = host(h_gpu)[:Rp]
-    close(bf(hg), bf(fw["h"]), what="h")
+    close(bf(hg), bf(fw["h"]), bf16=True, what="h")
     hq_ref, hs_ref = orc.quant_block(hg, 1, 128)          # the fused h-quantiser
     same_bits(host(B.hq)[:Rp], hq_ref, "hq = quant(h)")
     same_bits(host(B.hs)[:, :Rp].T, hs_ref, "hs = quant(h)")
@@ -89,13 +89,13 @@ def test_layer_parity(A, orc, case):
         gu = host(B.gu)[:Rp]
         gi = np.concatenate([gu[:, 256 * b:256 * b + 128] for b in range(I // 128)], axis=1)
         ui = np.concatenate([gu[:, 256 * b + 128:256 * b + 256] for b in range(I // 128)], axis=1)
-        close(bf(gi), fw["g"], what="g")
-        close(bf(ui), fw["u"], what="u")
+        close(bf(gi), bf(fw["g_b"]), bf16=True, what="g")
+        close(bf(ui), bf(fw["u_b"]), bf16=True, what="u")
 
     # ---- GEMM2 step on the GPU's hq
     Wq = fw["Wq"]
     Y_ref = OL.down_rows(host(B.hq)[:Rp], host(B.hs)[:, :Rp].T.copy(), fw["expert"], Wq[2])
-    close(bf(host(B.Y)[:Rp]), bf(Y_ref), what="Y")
+    close(bf(host(B.Y)[:Rp]), bf(Y_ref), bf16=True, what="Y")
 
     if not train:
         return
@@ -105,9 +105,12 @@ def test_layer_parity(A, orc, case):
 
     # ---- backward steps on the GPU's own upstream operands
     expert = fw["expert"]
-    dYr = OL.scaled_rows(dy, w, fw["pos"], Rp)   # bit-exact input of b2
+    # dY rows from the GPU's own routing weights (the same inputs): bit-exact
+    dYr = OL.scaled_rows(dy, host(B.w), fw["pos"], Rp)
     same_bits(host(B.dYb)[:Rp], dYr, "dY rows")
-    same_bits(host(B.dYq)[:Rp], bw["dYq"], "dYq")
+    dYq_ref, dYs_ref = orc.quant_block(dYr, 1, 128)
+    same_bits(host(B.dYq)[:Rp], dYq_ref, "dYq")
+    same_bits(host(B.dYs)[:, :Rp].T, dYs_ref, "dYs")
     dH = OL.dgrad_down(host(B.dYq)[:Rp], host(B.dYs)[:, :Rp].T.copy(), expert, Wq[2])
     gu = host(B.gu)[:Rp]
     g_b = np.concatenate([gu[:, 256 * b:256 * b + 128] for b in range(I // 128)], axis=1)
@@ -116,8 +119,8 @@ def test_layer_parity(A, orc, case):
     dGU = host(B.dGU)[:Rp]
     dG = np.concatenate([dGU[:, 256 * b:256 * b + 128] for b in range(I // 128)], axis=1)
     dU = np.concatenate([dGU[:, 256 * b + 128:256 * b + 256] for b in range(I // 128)], axis=1)
-    close(bf(dG), bf(dG_ref), what="dG")
-    close(bf(dU), bf(dU_ref), what="dU")
+    close(bf(dG), bf(dG_ref), bf16=True, what="dG")
+    close(bf(dU), bf(dU_ref), bf16=True, what="dU")
     q_ref, s_ref = orc.quant_block(dGU, 1, 128)     # the fused d[g|u] quantiser
     same_bits(host(B.dGUq)[:Rp], q_ref, "dGUq = quant(dGU)")
     same_bits(host(B.dGUs)[:, :Rp].T, s_ref, "dGUs = quant(dGU)")
@@ -131,12 +134,14 @@ def test_layer_parity(A, orc, case):
     dGs = dGUs[:, 0::2].copy()
     dUs = dGUs[:, 1::2].copy()
     dX_ref = OL.dgrad_gateup(dGq, dGs, dUq, dUs, expert, Wq[0], Wq[1])
-    close(bf(host(B.dX)[:Rp]), bf(dX_ref), what="dX")
+    close(bf(host(B.dX)[:Rp]), bf(dX_ref), bf16=True, what="dX")
     # b4 on the GPU's 128x1 operands
     hqT, hsT = host(B.hqT)[:, :Rp].T.copy(), host(B.hsT)[:Rp // 128]
     same_bits((hqT, hsT)[0], orc.quant_block(host(B.h)[:Rp], 128, 1)[0], "h 128x1 codes")
     dYqT, dYsT = host(B.dYqT)[:, :Rp].T.copy(), host(B.dYsT)[:Rp // 128]
-    same_bits(dYqT, bw["dYqT"], "dY 128x1 codes")
+    dYqT_ref, dYsT_ref = orc.quant_block(dYr, 128, 1)
+    same_bits(dYqT, dYqT_ref, "dY 128x1 codes")
+    same_bits(dYsT, dYsT_ref, "dY 128x1 scales")
     xqT, xsT = host(B.xqT)[:, :Rp].T.copy(), host(B.xsT)[:Rp // 128]
     offs = fw["offsets"]
     for e in range(E):
@@ -152,7 +157,7 @@ def test_layer_parity(A, orc, case):
     close(host(B.d_w), bw["d_w"], what="d_w")          # upstream of any re-quantisation
     close(host(B.d_logits), bw["dz"], what="d_logits")
     e2e = dict(max_abs_rms=MAX_ABS_RMS_E2E)
-    close(bf(host(B.dx)), bf(bw["dx"]), what="dx end to end", **e2e)
+    close(bf(host(B.dx)), bf(bw["dx"]), bf16=True, what="dx end to end", **e2e)
     dWg = np.concatenate([dWgu[:, 256 * b:256 * b + 128] for b in range(I // 128)], axis=1)
     dWu = np.concatenate([dWgu[:, 256 * b + 128:256 * b + 256] for b in range(I // 128)], axis=1)
     close(dWd, bw["dWd"], what="dW_down end to end", **e2e)
@@ -166,7 +171,9 @@ def test_layer_deterministic(A):
     outs = []
     for _ in range(2):
         d, W, B, h = _run_gpu(A, T, D, I, E, k, z, x, Wg, Wu, Wd, dy, train)
-        outs.append([host(t) for t in (B.y, B.dx, B.d_w, B.d_logits, B.dWd, B.dWgu, B.hq, B.dGUq)])
+        Rp = int(host(B.offsets)[E])  # rows past the last segment are never written
+        outs.append([host(t) for t in (B.y, B.dx, B.d_w, B.d_logits, B.dWd, B.dWgu)]
+                    + [host(B.hq)[:Rp], host(B.dGUq)[:Rp], host(B.Y)[:Rp], host(B.dX)[:Rp]])
     for a, b in zip(*outs):
         same_bits(a, b, "repeat run")
 
