@@ -132,6 +132,22 @@ int moe_permute(const int32_t *idx, const moe_dims *dims, int32_t *counts, int32
                 int32_t *pos, int32_t *src_idx, const uint16_t *x, uint8_t *xq, float *xs,
                 uint8_t *xqT, float *xsT, void *ws, size_t ws_bytes, void *stream);
 
+/* moe_permute without the caller-provided scratch, for callers that cannot
+ * allocate device memory (an engine step that has reserved all of HBM and
+ * forbids allocation while it runs; a plugin or custom-op host that passes
+ * only input and output tensors).  The pages have no counterpart: this is an
+ * interface variant, not a step of the method.  Same outputs as moe_permute
+ * without the 128x1 outputs.  The scratch is a fixed 1 MiB array inside the
+ * library, one per device that loads it, held until the process exits; a
+ * problem needing more (moe_permute_workspace_size() > 1 MiB) returns
+ * MOE_ERR_UNSUPPORTED.  The first call on a device looks up the array's
+ * address (make it before any stream capture); calls overlapping on the GPU
+ * share the array and race; entries outside [0,E) are dropped (pos = -1) but
+ * not reported through moe_get_status(). */
+int moe_permute_noalloc(const int32_t *idx, const moe_dims *dims, int32_t *counts, int32_t *offsets,
+                        int32_t *pos, int32_t *src_idx, const uint16_t *x, uint8_t *xq, float *xs,
+                        void *stream);
+
 /* ------------------------------------------------------------------------ */
 /* Block-scaled FP8 quantiser  [P4 §FP8 Training]                            */
 /* ------------------------------------------------------------------------ */

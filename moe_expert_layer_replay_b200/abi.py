@@ -20,7 +20,7 @@ EXPORTS = [
     "moe_rows_capacity", "moe_permute_workspace_size", "moe_strerror", "moe_get_status",
     "moe_set_wait_budget", "moe_route_topk", "moe_route_replay", "moe_permute",
     "moe_quant_fp8_block", "moe_quant_weights", "moe_grouped_gemm_fp8", "moe_combine",
-    "moe_combine_bwd", "moe_unpermute_reduce",
+    "moe_combine_bwd", "moe_unpermute_reduce", "moe_permute_noalloc",
 ]
 
 
@@ -66,6 +66,7 @@ def lib() -> ctypes.CDLL:
             "moe_route_topk": (ctypes.c_int, [P, D, P, P, P]),
             "moe_route_replay": (ctypes.c_int, [P, I32, I32, D, P, P, P, P, P]),
             "moe_permute": (ctypes.c_int, [P, D, P, P, P, P, P, P, P, P, P, P, SZ, P]),
+            "moe_permute_noalloc": (ctypes.c_int, [P, D, P, P, P, P, P, P, P, P]),
             "moe_quant_fp8_block": (ctypes.c_int, [P, I64, I64, I64, I32, I32, P, P, P, P, P]),
             "moe_quant_weights": (ctypes.c_int, [P, P, P, D, P, P, P, P, P, P, P, P, P]),
             "moe_grouped_gemm_fp8": (ctypes.c_int, [I32, D, P, ctypes.POINTER(GemmArgs), P]),
@@ -141,6 +142,12 @@ def permute(idx, d: Dims, counts, offsets, pos, src_idx, x, xq, xs, xqT, xsT, ws
     _check("moe_permute", lib().moe_permute(_p(idx), ctypes.byref(d), _p(counts), _p(offsets), _p(pos),
                                             _p(src_idx), _p(x), _p(xq), _p(xs), _p(xqT), _p(xsT), _p(ws),
                                             ws.numel() * ws.element_size(), _s(stream)))
+
+
+def permute_noalloc(idx, d: Dims, counts, offsets, pos, src_idx, x, xq, xs, stream=None):
+    """moe_permute with the library's own fixed scratch (no workspace argument)."""
+    _check("moe_permute_noalloc", lib().moe_permute_noalloc(_p(idx), ctypes.byref(d), _p(counts), _p(offsets),
+                                                            _p(pos), _p(src_idx), _p(x), _p(xq), _p(xs), _s(stream)))
 
 
 def quant_fp8_block(inp, rows, cols, ld, blk_r, blk_c, q, s, qT=None, sT=None, stream=None):
