@@ -128,14 +128,12 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, uint
     const long long t0 = clock64();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 31u) == 0) {  // the budget and the abort flag are checked every 32 polls
-            if (*abort_flag) return false;
-            if ((uint64_t)(clock64() - t0) > budget) {
-                *abort_flag = 1;
-                latch_status(status, MOE_ERR_TIMEOUT);
-                return false;
-            }
+        if ((uint64_t)(clock64() - t0) > budget) {
+            *abort_flag = 1;
+            latch_status(status, MOE_ERR_TIMEOUT);
+            return false;
         }
+        if ((it & 7u) == 0 && *abort_flag) return false;  // another role gave up
     }
 }
 

@@ -188,3 +188,27 @@ def test_wgrad_accumulates(A):
     layer.backward(B, dev(dy), W, router_logits=True)
     torch.cuda.synchronize()
     np.testing.assert_allclose(host(B.dWd), 2 * once, rtol=1e-6, atol=1e-12)
+
+
+def test_wait_budget_timeout_is_reported_and_recoverable(A):
+    """A wait budget too small for any real wait makes the GEMM's bounded
+    waits run out: the kernel latches MOE_ERR_TIMEOUT, drains its own copies
+    and MMAs, frees its tensor memory and returns; the context stays usable
+    and the next run with the default budget is correct."""
+    from moe_expert_layer_replay_b200 import layer
+    T, D, I, E, k, zipf, train = CASES["multi_tile"]
+    z, x, Wg, Wu, Wd, dy = _inputs(T, D, I, E, k, zipf, seed=8)
+    d, W, B, h = _run_gpu(A, T, D, I, E, k, z, x, Wg, Wu, Wd, dy, False)
+    ref_hq = host(B.hq).copy()
+    Rp = int(host(B.offsets)[E])
+    try:
+        A.set_wait_budget(1)
+        A.grouped_gemm_fp8(A.GEMM_GATEUP_SILU, d, B.offsets, B.xq, B.xs, W.wgu_q, W.wgu_s,
+                           out_q=B.hq, out_s=B.hs)
+        st = A.get_status()
+    finally:
+        A.set_wait_budget(0)
+    assert st == A.TIMEOUT, A.strerror(st)
+    A.grouped_gemm_fp8(A.GEMM_GATEUP_SILU, d, B.offsets, B.xq, B.xs, W.wgu_q, W.wgu_s, out_q=B.hq, out_s=B.hs)
+    assert A.get_status() == A.OK
+    same_bits(host(B.hq)[:Rp], ref_hq[:Rp], "after a timed-out run")
