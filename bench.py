@@ -38,6 +38,21 @@ METRIC = "MoE-layer tokens/s; grouped FP8 GEMM TFLOP/s as % of dense FP8 peak"
 UNIT = "tokens/s"
 FP8_OVER_BF16 = 2.0  # nominal dense ratio (4.5 / 2.25 PFLOP/s)
 
+# DRAM traffic (read + write bytes) of one gate/up GEMM launch of this
+# workload, from the ncu capture summarised in profiles/grouped_gemm_replay_ncu.md.
+# Valid only for the kernel sources it was taken on: reported as null as soon
+# as their hash differs.
+GEMM1_TRAFFIC = {"sources_sha256_16": "b9c29c9f2af72501", "bytes": 356.882432e6}
+
+
+def _gemm_sources_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("gemm_sm100.cu", "common.cuh"):
+        with open(os.path.join(ROOT, "moe_expert_layer_replay_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
 
 def _peaks():
     try:
@@ -306,7 +321,9 @@ def run_ours(args, wl_name):
                        "parallelism": "replicas" if world > 1 else "single GPU"},
             "roofline": {"bound": "tensor", "kernel": "grouped_gemm gate/up + SiLU + h-quant",
                          "achieved": achieved, "peak": fp8_peak, "unit": "TFLOP/s", "frac": achieved / fp8_peak,
-                         "traffic": None,
+                         "traffic": (GEMM1_TRAFFIC["bytes"] if _gemm_sources_hash() == GEMM1_TRAFFIC["sources_sha256_16"]
+                                     else None),
+                         "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
                          "peak_note": f"fp8 dense = {FP8_OVER_BF16} x {src} bf16 burst {bf16_tf} TFLOP/s",
                          "algorithmic": f"2*R*D*2I = {g1_flop:.4g} FLOP per launch (R = T*k routed rows)",
                          "avg_launch_ms": g1_avg},
