@@ -69,25 +69,36 @@ def _workload_desc(wl):
 
 
 class Clocks:
-    """nvidia-smi sampling of SM clocks and throttle reasons during a region."""
+    """nvidia-smi sampling (every 20 ms, with timestamps) of SM clocks and
+    throttle reasons; stop() keeps the samples taken between mark() and the
+    stop call (warm-up plus the timed steps: the same work)."""
 
     def __init__(self, index: int, path: str):
         self.path = path
         self.p = None
-        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+        self.t0 = None
+        q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
         try:
             self.f = open(path, "w")
             self.p = subprocess.Popen(["nvidia-smi", f"--id={index}", f"--query-gpu={q}",
-                                       "--format=csv,noheader,nounits", "-lms", "200"],
+                                       "--format=csv,noheader,nounits", "-lms", "20"],
                                       stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.5)  # let the sampler start before the region of interest
         except Exception:
             self.p = None
 
+    def mark(self):
+        import datetime
+        self.t0 = datetime.datetime.now()
+
     def stop(self):
+        import datetime
         if self.p is None:
             return None
+        t1 = datetime.datetime.now()
+        time.sleep(0.1)
         self.p.terminate()
         try:
             self.p.wait(timeout=5)
@@ -98,20 +109,50 @@ class Clocks:
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in open(self.path):
             parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9:
+            if len(parts) < 10:
                 continue
             try:
-                sm.append(float(parts[1]))
-                mx.append(float(parts[2]))
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f")
+                if self.t0 is not None and not (self.t0 <= ts <= t1):
+                    continue
+                sm.append(float(parts[2]))
+                mx.append(float(parts[3]))
             except ValueError:
                 continue
-            for n, v in zip(names, parts[5:9]):
+            for n, v in zip(names, parts[6:10]):
                 if v.lower() == "active":
                     reasons.add(n)
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "window": "warm-up and timed steps"}
+
+
+# --------------------------------------------------------------------------
+# multi-rank plumbing (replicas: no data-path collective)
+# --------------------------------------------------------------------------
+
+def replica_seed(seed: int, rank: int) -> int:
+    """Each rank draws its own batch of the workload."""
+    return seed + rank
+
+
+def reduce_max(value: float) -> float:
+    """Max over ranks (the step time every rank must wait for); identity on
+    one process.  Uses the process group's backend (NCCL: a CUDA tensor)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(value)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_rate(world: int, units_per_rank: float, max_seconds: float) -> float:
+    """Whole-job throughput: the units all ranks processed / the slowest rank's time."""
+    return world * units_per_rank / max_seconds
 
 
 # --------------------------------------------------------------------------
@@ -197,7 +238,7 @@ def run_ours(args, wl_name):
         dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local))
     abi.lib()
 
-    inp = make_inputs(wl_name, seed=args.seed + rank)
+    inp = make_inputs(wl_name, seed=replica_seed(args.seed, rank))
     wl = inp["workload"]
     d = abi.dims(wl.T, wl.D, wl.I, wl.E, wl.k)
     dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16) if a.dtype == np.uint16 else
@@ -231,6 +272,9 @@ def run_ours(args, wl_name):
 
     launches_per_step = wl.L * (1 + 5 + 1 + 1 + 1)  # replay, permute (count/scan/place/quant/pad), 2 GEMMs, combine
 
+    clocks = Clocks(local, os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv")) \
+        if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else Clocks(local, f"/tmp/moe_clocks_{rank}.csv")
+    clocks.mark()
     for _ in range(max(3, args.warmup)):
         step(False)
     torch.cuda.synchronize()
@@ -243,8 +287,6 @@ def run_ours(args, wl_name):
             dist.barrier()
         torch.cuda.synchronize()
 
-    clocks = Clocks(local, os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv")) \
-        if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else Clocks(local, f"/tmp/moe_clocks_{rank}.csv")
     barrier()
     step_ms = []
     for _ in range(args.steps):
@@ -258,13 +300,9 @@ def run_ours(args, wl_name):
     clk = clocks.stop()
     step_ms = [a.elapsed_time(b) for a, b in step_ms]
     g1_ms = [a.elapsed_time(b) for a, b in gemm1_events]
-    tot_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([tot_ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        tot_ms = float(t.item())
+    tot_ms = reduce_max(sum(step_ms))
     ms_per_step = tot_ms / args.steps
-    value = world * wl.L * wl.T * args.steps / (tot_ms / 1e3)
+    value = aggregate_rate(world, wl.L * wl.T * args.steps, tot_ms / 1e3)
 
     # ---------------- end to end through the C ABI with host buffers
     xh = torch.from_numpy(inp["x"].view(np.int16)).pin_memory()
@@ -291,12 +329,8 @@ def run_ours(args, wl_name):
         e2e_step()
     e1.record(stream)
     barrier()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_val = world * wl.L * wl.T * args.steps / (e2e_ms / 1e3)
+    e2e_ms = reduce_max(e0.elapsed_time(e1))
+    e2e_val = aggregate_rate(world, wl.L * wl.T * args.steps, e2e_ms / 1e3)
     h2d = xh.numel() * 2 + ph.numel() * 4 + wh.numel() * 4
     d2h = yh.numel() * 2
 
