@@ -506,16 +506,23 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     if (kEpi == EPI_SILU) return (c < 2) ? (64 * h + 32 * c) : (128 + 64 * h + 32 * (c - 2));
                     return 128 * h + 32 * c;
                 };
-                // TMEM reads pipelined one chunk ahead of the FMAs; the buffer
-                // goes back to the MMA as soon as the last read has landed
+                // TMEM reads two chunks (64 columns) at a time with one wait per
+                // pair; the buffer goes back to the MMA as soon as the second
+                // pair has landed, before its FMAs
                 uint32_t ra[32], rb[32];
-                MOE_TMEM_LD32(cbase + col_of(0), ra);
-                tmem_wait_ld();
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     uint32_t *cur = (c & 1) ? rb : ra;
-                    uint32_t *nxt = (c & 1) ? ra : rb;
-                    if (c + 1 < 4) MOE_TMEM_LD32(cbase + col_of(c + 1), nxt);
+                    if ((c & 1) == 0) {
+                        MOE_TMEM_LD32(cbase + col_of(c), ra);
+                        MOE_TMEM_LD32(cbase + col_of(c + 1), rb);
+                        tmem_wait_ld();
+                        if (c == 2) {
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(bar_tempty + 8 * buf);
+                        }
+                    }
                     if (kWgrad) {
                         const float *cs = d + 256 + 128 * h + 32 * c;
 #pragma unroll
@@ -529,12 +536,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                             ffma2(acc[32 * c + i], acc[32 * c + i + 1], __uint_as_float(cur[i]),
                                   __uint_as_float(cur[i + 1]), sc, sc);
                     }
-                    if (c + 1 < 4) tmem_wait_ld();
-                    if (c == 2) {
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(bar_tempty + 8 * buf);
-                    }
+
                 }
                 buf ^= 1;
                 if (buf == 0) bphase ^= 1;
