@@ -50,21 +50,38 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr uint64_t DRAIN_BUDGET = 1ull << 28;
 constexpr int PF = 3;  // scale prefetch depth (K blocks)
 // smem: operand ring | barriers (full[4], empty[4], tfull[2], tempty[2], drain, epi) |
-// tmem slot | abort flag | offsets[257] | amax exchange [2][2][128] |
-// scale ring [PF][3][256] fp32 (per epilogue thread: row scale, weight/column
-// scale, second weight scale) | bf16 output staging [8 warps][32 rows][80 B]
+// tmem slot | abort flag | offsets[257] | then, 1024-aligned, a region whose
+// use depends on the epilogue:
+//   SILU   amax exchange [2][2][128] fp32 | h-code store buffers [8 warps][32 rows][64 B]
+//   BF16   output store buffers [8 warps][2][32 rows][64 B]
+//   WGRAD  column-scale ring [PF][3][256] fp32 (per epilogue thread: row scale,
+//          column scale, spare)
+//   DSILU  unused
+// Store buffers are read by TMA stores (32 rows x 64 bytes boxes, no swizzle).
 constexpr int OFF_BAR = STAGES * STAGE_BYTES;
 constexpr int OFF_TMEM_SLOT = OFF_BAR + 16 * 8;
 constexpr int OFF_ABORT = OFF_TMEM_SLOT + 4;
 constexpr int OFF_OFFSETS = OFF_BAR + 256;
-constexpr int OFF_AMAX = OFF_OFFSETS + 1040;
-constexpr int OFF_RING = OFF_AMAX + 2 * 2 * 128 * 4;
-constexpr int STAGE_ROW = 80;  // 64 B of bf16 + 16 B pad: conflict-free 16-byte rows
-constexpr int OFF_STAGE = OFF_RING + PF * 3 * 256 * 4;
-constexpr int SMEM_BYTES = OFF_STAGE + 8 * 32 * STAGE_ROW + 1024;  // + alignment slack
-static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+constexpr int OFF_EPI = (OFF_OFFSETS + 1040 + 1023) / 1024 * 1024;
+constexpr int OFF_AMAX = OFF_EPI;
+constexpr int OFF_RING = OFF_EPI;
+constexpr int TSTORE_BUF = 32 * 64;
+constexpr int OFF_TSTORE_SILU = OFF_EPI + 2 * 2 * 128 * 4;
+constexpr int OFF_TSTORE_BF16 = OFF_EPI;
 
 enum Epi { EPI_SILU = 0, EPI_BF16 = 1, EPI_DSILU = 2, EPI_WGRAD = 3 };
+
+template <int kEpi>
+constexpr int smem_bytes()
+{
+    return 1024 + (kEpi == EPI_SILU   ? OFF_TSTORE_SILU + 8 * TSTORE_BUF
+                   : kEpi == EPI_BF16 ? OFF_TSTORE_BF16 + 8 * 2 * TSTORE_BUF
+                   : kEpi == EPI_WGRAD ? OFF_RING + PF * 3 * 256 * 4
+                                       : OFF_EPI);  // + alignment slack
+}
+static_assert(smem_bytes<EPI_SILU>() <= 232448 && smem_bytes<EPI_BF16>() <= 232448 &&
+                  smem_bytes<EPI_WGRAD>() <= 232448 && smem_bytes<EPI_DSILU>() <= 232448,
+              "shared memory budget");
 
 struct Args {
     const int32_t *offsets;
@@ -181,6 +198,20 @@ __device__ __forceinline__ void ffma2(float &a0, float &a1, float p0, float p1, 
         : "f"(p0), "f"(p1), "f"(s0), "f"(s1));
 }
 
+// TMA store of a 2D box from shared memory (bulk-group completion).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t src, int32_t c0, int32_t c1)
+{
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(src), "r"(c0), "r"(c1)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+template <int n>
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(n) : "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
@@ -285,7 +316,7 @@ __device__ __forceinline__ Tile tile_of(int t, const Args &p, const int *offs_s)
 template <int kEpi>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                    const Args p)
+                    const __grid_constant__ CUtensorMap tmC, const Args p)
 {
     constexpr bool kWgrad = (kEpi == EPI_WGRAD);
     extern __shared__ uint8_t smem_raw[];
@@ -571,9 +602,19 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 if (!epi_sync()) break;
                 amax = fmaxf(ax[row], ax[128 + row]);
                 const float s = block_scale(amax);
-                uint8_t *hq = p.out_q + r * I + icol;
+                // this warp's 32 rows x 64 codes leave through one TMA store
+                uint8_t *sb = smem + OFF_TSTORE_SILU + ew * TSTORE_BUF;
+                if (lane == 0) bulk_wait_read<0>();  // the previous tile's store has read sb
+                __syncwarp();
 #pragma unroll
-                for (int i0 = 0; i0 < 64; i0 += 16) *reinterpret_cast<uint4 *>(hq + i0) = quant16(&acc[i0], s);
+                for (int i0 = 0; i0 < 64; i0 += 16)
+                    *reinterpret_cast<uint4 *>(sb + lane * 64 + i0) = quant16(&acc[i0], s);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(&tmC, smem_u32(sb), (int32_t)icol, x.m0 + 32 * q);
+                    bulk_commit();
+                }
                 if (h == 0) p.out_s[(int64_t)x.nt * p.R_cap + r] = s;
                 if (p.out_bf16) {
                     uint16_t *hb = p.out_bf16 + r * I + icol;
@@ -581,25 +622,24 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     for (int i0 = 0; i0 < 64; i0 += 8) *reinterpret_cast<uint4 *>(hb + i0) = pack8(&acc[i0]);
                 }
             } else if (kEpi == EPI_BF16) {
-                // through a per-warp smem tile, so that each store instruction
-                // writes 8 rows x 64 contiguous bytes instead of 32 scattered 16 B
+                // 32-column chunks through two per-warp smem buffers, written to
+                // global memory by TMA stores that run while the warp moves on
                 const int64_t c0 = (int64_t)x.n0 + 128 * h;
                 if (c0 < p.N) {
-                    uint8_t *stg = smem + OFF_STAGE + ew * 32 * STAGE_ROW;
-                    const int64_t rbase = (int64_t)x.m0 + 32 * q;
 #pragma unroll
                     for (int ch = 0; ch < 4; ++ch) {
-                        uint4 *w = reinterpret_cast<uint4 *>(stg + lane * STAGE_ROW);
+                        uint8_t *buf = smem + OFF_TSTORE_BF16 + (ew * 2 + (ch & 1)) * TSTORE_BUF;
+                        if (lane == 0) bulk_wait_read<1>();  // the store that last read buf is done
+                        __syncwarp();
+                        uint4 *w = reinterpret_cast<uint4 *>(buf + lane * 64);
 #pragma unroll
                         for (int j = 0; j < 4; ++j) w[j] = pack8(&acc[32 * ch + 8 * j]);
+                        fence_proxy_async_smem();
                         __syncwarp();
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const int rr = (lane & 7) + 8 * i, pc = lane >> 3;
-                            const uint4 v = *reinterpret_cast<const uint4 *>(stg + rr * STAGE_ROW + pc * 16);
-                            *reinterpret_cast<uint4 *>(p.out_bf16 + (rbase + rr) * p.N + c0 + 32 * ch + 8 * pc) = v;
+                        if (lane == 0) {
+                            tma_store_2d(&tmC, smem_u32(buf), (int32_t)(c0 + 32 * ch), x.m0 + 32 * q);
+                            bulk_commit();
                         }
-                        __syncwarp();
                     }
                 }
             } else if (kEpi == EPI_DSILU) {
@@ -668,6 +708,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             }
         }
         cp_async_wait<0>();  // no copy into shared memory outlives the CTA
+        if ((kEpi == EPI_SILU || kEpi == EPI_BF16) && lane == 0) bulk_wait_all();  // every TMA store has completed
     }
     tc_fence_before();
     __syncthreads();
@@ -707,6 +748,23 @@ static bool make_map(CUtensorMap *map, const void *base, uint64_t cols, uint64_t
     return r == CUDA_SUCCESS;
 }
 
+// Row-major [rows][cols] output of 1- or 2-byte elements, boxes of 32 rows x
+// 64 bytes, no swizzle (TMA stores of the SiLU and bf16 epilogues).
+static bool make_store_map(CUtensorMap *map, void *base, uint64_t cols, uint64_t rows, int esize)
+{
+    auto fn = get_encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * esize};
+    cuuint32_t box[2] = {(cuuint32_t)(64 / esize), 32};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, esize == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base,
+                    dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 static int sm_count()
 {
     int dev = 0, n = 0;
@@ -716,17 +774,17 @@ static int sm_count()
 }
 
 template <int kEpi>
-static int launch_one(const CUtensorMap &a, const CUtensorMap &b, const gemm::Args &args, int grid,
-                      cudaStream_t s)
+static int launch_one(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &c, const gemm::Args &args,
+                      int grid, cudaStream_t s)
 {
     static bool configured = false;  // per process; attribute is per function
     if (!configured) {
         if (cudaFuncSetAttribute(gemm::grouped_gemm_kernel<kEpi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 gemm::SMEM_BYTES) != cudaSuccess)
+                                 gemm::smem_bytes<kEpi>()) != cudaSuccess)
             return MOE_ERR_CUDA;
         configured = true;
     }
-    gemm::grouped_gemm_kernel<kEpi><<<grid, gemm::NUM_THREADS, gemm::SMEM_BYTES, s>>>(a, b, args);
+    gemm::grouped_gemm_kernel<kEpi><<<grid, gemm::NUM_THREADS, gemm::smem_bytes<kEpi>(), s>>>(a, b, c, args);
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -778,13 +836,17 @@ int launch_grouped_gemm(int op, const moe_dims &d, int64_t R_cap, const int32_t 
         return MOE_ERR_INVALID_ARG;
     }
     if (!ok) return MOE_ERR_CUDA;
+    CUtensorMap mC = mA;  // output map of the epilogues that store through TMA
+    if (op == MOE_GEMM_GATEUP_SILU) ok = make_store_map(&mC, g.out_q, a.N / 2, R_cap, 1);
+    if (op == MOE_GEMM_DOWN || op == MOE_GEMM_DGRAD_GATEUP) ok = make_store_map(&mC, g.out_bf16, a.N, R_cap, 2);
+    if (!ok) return MOE_ERR_CUDA;
     const int grid = sm_count();
     switch (op) {
-    case MOE_GEMM_GATEUP_SILU: return launch_one<gemm::EPI_SILU>(mA, mB, a, grid, s);
+    case MOE_GEMM_GATEUP_SILU: return launch_one<gemm::EPI_SILU>(mA, mB, mC, a, grid, s);
     case MOE_GEMM_DOWN:
-    case MOE_GEMM_DGRAD_GATEUP: return launch_one<gemm::EPI_BF16>(mA, mB, a, grid, s);
-    case MOE_GEMM_DGRAD_DOWN_SILU: return launch_one<gemm::EPI_DSILU>(mA, mB, a, grid, s);
-    default: return launch_one<gemm::EPI_WGRAD>(mA, mB, a, grid, s);
+    case MOE_GEMM_DGRAD_GATEUP: return launch_one<gemm::EPI_BF16>(mA, mB, mC, a, grid, s);
+    case MOE_GEMM_DGRAD_DOWN_SILU: return launch_one<gemm::EPI_DSILU>(mA, mB, mC, a, grid, s);
+    default: return launch_one<gemm::EPI_WGRAD>(mA, mB, mC, a, grid, s);
     }
 }
 
