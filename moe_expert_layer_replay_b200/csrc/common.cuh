@@ -58,39 +58,28 @@ __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi)
 __device__ __forceinline__ float block_scale(float amax) { return __fdiv_rn(amax, 448.0f); }
 
 // The e4m3 code of the correctly rounded quotient q = RN_fp32(x / s),
-// without a divide per element.
+// without a divide per element and without a branch.
 //
-// With r = RN(1/s), q' = RN(x * r) is within 2^-23 relative of x/s, so within
-// 2.5 fp32 ulps of q.  e4m3 (3 mantissa bits) rounds q and q' to different
-// codes only if an e4m3 rounding midpoint M lies between them.  In e4m3's
-// normal range a midpoint is an fp32 value whose 20 low mantissa bits are
-// 0x80000; q' is "near" when those bits are within 4 of it.  Below 2^-6
-// (e4m3's subnormal grid, step 2^-9) every element is treated as near.
+// With r = RN(1/s), q' = RN(x * r) = (x/s)(1 + d), |d| < 3 * 2^-24, so q' is
+// within 3 fp32 ulps of q.  e4m3 (3 mantissa bits) rounds q and q' to
+// different codes only if an e4m3 rounding midpoint M lies between them or on
+// one of them.  In e4m3's normal range a midpoint is an fp32 value whose 20
+// low mantissa bits are 0x80000; q' is "near" when those bits are within 4 of
+// it.  Below 2^-6 (e4m3's subnormal grid, step 2^-9) the midpoints are the
+// odd multiples of 2^-10; adding 2^-6 maps them onto the midpoints of the
+// binade [2^-6, 2^-5) (same step), where the same bit test applies (the
+// addition's rounding adds at most half an ulp of the window).
 //
-// A near element is decided exactly against the midpoint M of its e4m3 cell:
-// q > M iff x/s > M + u/2, q < M iff x/s < M - u/2, else q == M (u = fp32 ulp
-// of M; M has 4 significant bits, so ties at M +- u/2 round to M).  The sign
-// of x - (M +- u/2) * s is exact in fp64: the product has 49 significant bits.
-// The element then converts through M (tie: even code) or its fp32 neighbour
-// on the decided side, which e4m3 rounds like q.  No midpoint is ever
-// decided by an approximation.
-__device__ __forceinline__ float near_midpoint_exact(float x, float s, float qp)
-{
-    const float aq = fabsf(qp);
-    const uint32_t b = __float_as_uint(aq);
-    const float M = (b < 0x3c800000u) ? (floorf(aq * 512.0f) + 0.5f) * (1.0f / 512.0f)
-                                      : __uint_as_float((b & 0xfff00000u) | 0x00080000u);
-    const double half_ulp = (double)__uint_as_float(__float_as_uint(M) & 0x7f800000u) * 0x1p-24;
-    const double xd = (double)fabsf(x), sd = (double)s;
-    float v;
-    if (xd - ((double)M + half_ulp) * sd > 0.0) v = __uint_as_float(__float_as_uint(M) + 1u);
-    else if (xd - ((double)M - half_ulp) * sd < 0.0) v = __uint_as_float(__float_as_uint(M) - 1u);
-    else v = M;
-    return copysignf(v, x);
-}
-
-// IEEE division for a whole group; only for scales whose reciprocal is not
-// finite (amax below about 1.5e-36), kept out of line.
+// A near element is decided exactly against M: q > M iff x/s > M + u/2,
+// q < M iff x/s < M - u/2, else q == M (u = fp32 ulp of M; M has 4 significant
+// bits, so its last fp32 mantissa bit is 0 and ties at M +- u/2 round to M;
+// the one midpoint that is a power of two, 2^-10, ties down to the code 0
+// either way).  For a near element x - M*s is a small multiple of the grid of
+// M*s (at most 11 significant bits), so fma(-M, s, |x|) is that difference
+// exactly, and it is compared with the exact u/2 * s.  This needs
+// s >= 2^-100 (no underflow in the grid or in u/2 * s); smaller scales take
+// the IEEE division.  The element converts through M, or its fp32 neighbour
+// on the decided side, which e4m3 rounds like q.
 template <int n>
 struct Floats {
     float v[n];
@@ -110,7 +99,7 @@ template <int n>
 __device__ __forceinline__ void quotients(const float *v, float s, float *q)
 {
     const float r = __frcp_rn(s);
-    if (!(r <= 3.0e38f)) {
+    if (!(r <= 0x1p100f)) {  // s below about 2^-100: IEEE division, out of line
         Floats<n> x;
 #pragma unroll
         for (int i = 0; i < n; ++i) x.v[i] = v[i];
@@ -119,12 +108,20 @@ __device__ __forceinline__ void quotients(const float *v, float s, float *q)
         for (int i = 0; i < n; ++i) q[i] = e.v[i];
         return;
     }
+    const float s24 = s * 0x1p-24f;  // u/2 * s = s24 * 2^exponent(M), exact
 #pragma unroll
     for (int i = 0; i < n; ++i) {
-        q[i] = __fmul_rn(v[i], r);
-        const uint32_t b = __float_as_uint(q[i]) & 0x7fffffffu;
-        const int low = (int)(b & 0xfffffu) - 0x80000;
-        if ((b < 0x3c800000u && b != 0u) || (low >= -4 && low <= 4)) q[i] = near_midpoint_exact(v[i], s, q[i]);
+        const float qp = __fmul_rn(v[i], r);
+        const uint32_t b = __float_as_uint(qp) & 0x7fffffffu;
+        const bool sub = b < 0x3c800000u;
+        const uint32_t y = sub ? __float_as_uint(__fadd_rn(__uint_as_float(b), 0x1p-6f)) : b;
+        const bool near = ((y - 0x7fffcu) & 0xfffffu) <= 8u;
+        const float My = __uint_as_float((y & 0xfff00000u) | 0x00080000u);
+        const float M = sub ? __fsub_rn(My, 0x1p-6f) : My;
+        const float c = __fmul_rn(s24, __uint_as_float(__float_as_uint(M) & 0x7f800000u));
+        const float e = __fmaf_rn(-M, s, fabsf(v[i]));
+        const uint32_t mb = __float_as_uint(M) + (e > c ? 1u : 0u) - (e < -c ? 1u : 0u);
+        q[i] = near ? __uint_as_float(mb | (__float_as_uint(qp) & 0x80000000u)) : qp;
     }
 }
 
