@@ -20,14 +20,22 @@ __device__ __forceinline__ void latch_status(int *status, int code)
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
+// fp32 -> bf16 bits, round to nearest even, on the integer pipe: finite
+// values round as the IEEE conversion does (overflow goes to infinity); a NaN
+// becomes the canonical bf16 NaN 0x7fff.
 __device__ __forceinline__ uint32_t bf16_bits_rn(float f)
 {
-    return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(f));
+    const uint32_t u = __float_as_uint(f);
+    if ((u & 0x7fffffffu) > 0x7f800000u) return 0x7fffu;
+    return (u + 0x7fffu + ((u >> 16) & 1u)) >> 16;
 }
 
+// Two fp32 -> packed bf16x2 (lo in the low half), round to nearest even.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 {
-    return bf16_bits_rn(lo) | (bf16_bits_rn(hi) << 16);
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
 }
 
 // 8 bf16 (one 16-byte vector) -> 8 floats.

@@ -298,3 +298,31 @@ def test_quant_exhaustive_bf16(A, orc, blk):
         oq, os_ = orc.quant_block(x, 128, 128)
         same_bits(host(q), oq, "codes")
         same_bits(host(s), os_, "scales")
+
+
+def test_quant_scale_sweep_bf16(A, orc):
+    """Every bf16 mantissa against every block scale from the subnormal range
+    up: block b holds its planted amax m_b * 2^e_b and the 128 bf16 mantissas
+    spread over the 20 binades below it.  Amax mantissas include 1.75 and 1.5,
+    for which many quotients fall exactly on e4m3 rounding midpoints (the ties
+    the quantiser must decide exactly); the sweep crosses the scale range where
+    the kernel switches from its reciprocal path to IEEE division."""
+    rng = np.random.default_rng(11)
+    mants = 1.0 + np.arange(128) / 128.0
+    amax_m = np.array([1.0, 1.5, 1.75, 1.25, 1.9921875, 1.0078125, 1.375, 1.625])
+    blocks = []
+    for e in range(-126, 121):
+        for am in amax_m:
+            shift = rng.integers(0, 21, 128)
+            sign = rng.choice([-1.0, 1.0], 128)
+            v = sign * rng.permutation(mants) * np.ldexp(1.0, e - shift)
+            v[rng.integers(0, 128)] = am * np.ldexp(1.0, e) * rng.choice([-1.0, 1.0])
+            blocks.append(v)
+    x = orc.bf16_round(np.stack(blocks))  # values below the bf16 range flush to signed zero
+    rows, cols = x.shape
+    q = torch.empty(rows, cols, dtype=torch.uint8, device="cuda")
+    s = torch.empty(1, rows, dtype=torch.float32, device="cuda")
+    A.quant_fp8_block(dev(x), rows, cols, cols, 1, 128, q, s)
+    oq, os_ = orc.quant_block(x, 1, 128)
+    same_bits(host(s).T, os_, "scales")
+    same_bits(host(q), oq, "codes")
