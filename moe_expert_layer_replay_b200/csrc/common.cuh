@@ -183,6 +183,9 @@ size_t permute_ws_bytes(int T, int k, int E);
 int launch_quant_1x128(const uint16_t *in, int64_t ld, int64_t rows, int64_t cols,
                        const int32_t *pos, int k, uint8_t *q, int64_t ldq, float *sc,
                        int64_t ld_s, cudaStream_t s);
+int launch_dispatch_quant(const uint16_t *x, int64_t T, int64_t D, const int32_t *pos, int k, uint8_t *xq,
+                          float *xs, int64_t R_cap, const int32_t *counts, const int32_t *offsets, int E,
+                          cudaStream_t s);
 int launch_quant_rows128(const uint16_t *in, int64_t ld, const int32_t *src_idx, int k,
                          int64_t rows, int64_t cols, int64_t ld_rows, uint8_t *qT, float *sT,
                          cudaStream_t s);

@@ -140,9 +140,7 @@ int moe_permute(const int32_t *idx, const moe_dims *d, int32_t *counts, int32_t 
     st = moe::launch_permute_index(idx, d->T, d->k, d->E, d->align, counts, offsets, pos, src_idx,
                                    R_cap, ws, sp, s);
     if (st || !x) return st;
-    st = moe::launch_quant_1x128(x, d->D, d->T, d->D, pos, d->k, xq, d->D, xs, R_cap, s);
-    if (st) return st;
-    st = moe::launch_pad_rows(counts, offsets, d->E, d->D, R_cap, xq, xs, nullptr, s);
+    st = moe::launch_dispatch_quant(x, d->T, d->D, pos, d->k, xq, xs, R_cap, counts, offsets, d->E, s);
     if (st || !xqT) return st;
     return moe::launch_quant_rows128(x, d->D, src_idx, d->k, R_cap, d->D, R_cap, xqT, xsT, s);
 }

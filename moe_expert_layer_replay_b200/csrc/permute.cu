@@ -7,7 +7,8 @@
 // with every expert's segment padded to a multiple of `align` rows.
 //
 // Three deterministic passes (no global atomics, so the result never depends
-// on scheduling):
+// on scheduling; the rows of src_idx that no entry fills are set to -1 by the
+// place pass):
 //   count: block b counts its chunk of entries per expert (shared atomics);
 //   scan:  per expert, an exclusive scan of the block counts (block bases),
 //          totals, then padded offsets;
@@ -64,22 +65,40 @@ __global__ void __launch_bounds__(256) perm_scan_kernel(const int32_t *__restric
         padded[e] = (run + align - 1) / align * align;
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-        int acc = 0;
-        offsets[0] = 0;
-        for (int i = 0; i < E; ++i) {
-            acc += padded[i];
-            offsets[i + 1] = acc;
+    if (threadIdx.x < 32) {  // exclusive scan of the padded sizes, 32 experts per step
+        const int lane = threadIdx.x;
+        int carry = 0;
+        for (int e0 = 0; e0 < E; e0 += 32) {
+            const int v = e0 + lane < E ? padded[e0 + lane] : 0;
+            int x = v;
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const int y = __shfl_up_sync(kFull, x, d);
+                if (lane >= d) x += y;
+            }
+            if (e0 + lane < E) offsets[e0 + lane] = carry + x - v;
+            carry += __shfl_sync(kFull, x, 31);
         }
+        if (lane == 0) offsets[E] = carry;
     }
 }
 
 __global__ void __launch_bounds__(256) perm_place_kernel(const int32_t *__restrict__ idx, int64_t n,
                                                          int E, const int32_t *__restrict__ blkbase,
                                                          const int32_t *__restrict__ offsets,
+                                                         const int32_t *__restrict__ counts, int64_t R_cap,
                                                          int32_t *__restrict__ pos,
                                                          int32_t *__restrict__ src_idx, int *status)
 {
+    // rows no entry fills: expert e's padding goes to block e % gridDim.x;
+    // the rows past offsets[E] are shared by all blocks
+    for (int e = blockIdx.x; e < E; e += gridDim.x)
+        for (int64_t r = (int64_t)offsets[e] + counts[e] + threadIdx.x; r < offsets[e + 1]; r += blockDim.x)
+            src_idx[r] = -1;
+    for (int64_t r = (int64_t)offsets[E] + (int64_t)blockIdx.x * blockDim.x + threadIdx.x; r < R_cap;
+         r += (int64_t)gridDim.x * blockDim.x)
+        src_idx[r] = -1;
+    if (n == 0) return;
     extern __shared__ int whist[];  // [kPlaceWarps][E]
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     for (int i = threadIdx.x; i < kPlaceWarps * E; i += blockDim.x) whist[i] = 0;
@@ -132,16 +151,13 @@ int launch_permute_index(const int32_t *idx, int T, int k, int E, int align, int
     int nblk = (int)((n + kChunk - 1) / kChunk);
     int32_t *blkcnt = (int32_t *)ws;
     int32_t *blkbase = blkcnt + (int64_t)(nblk ? nblk : 1) * E;
-    if (cudaMemsetAsync(src_idx, 0xff, (size_t)R_cap * sizeof(int32_t), s) != cudaSuccess)
-        return MOE_ERR_CUDA;
     if (nblk > 0) {
         perm_count_kernel<<<nblk, 256, E * sizeof(int), s>>>(idx, n, E, blkcnt);
     }
     perm_scan_kernel<<<1, 256, 0, s>>>(blkcnt, nblk, E, align, blkbase, counts, offsets);
-    if (nblk > 0) {
-        perm_place_kernel<<<nblk, 32 * kPlaceWarps, kPlaceWarps * E * sizeof(int), s>>>(
-            idx, n, E, blkbase, offsets, pos, src_idx, status);
-    }
+    // place also writes -1 to the rows of src_idx that no entry fills
+    perm_place_kernel<<<nblk > 0 ? nblk : 1, 32 * kPlaceWarps, kPlaceWarps * E * sizeof(int), s>>>(
+        idx, n, E, blkbase, offsets, counts, R_cap, pos, src_idx, status);
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

@@ -13,20 +13,41 @@ namespace moe {
 // ---------------------------------------------------------------------------
 // 1x128 blocks along a row, optionally scattered to k permuted rows.
 // One warp per input row; lane l covers 16 columns of each 512-column step,
-// so 8 lanes make one 128-block (amax by a 3-step xor butterfly).
+// so 8 lanes make one 128-block (amax by a 3-step xor butterfly).  The loads
+// of up to four steps (2048 columns) are issued before any is used.
 // Destination rows: pos == nullptr -> the row itself (k must be 1);
 // otherwise row t goes to pos[t*k + j] for each j with pos >= 0.
 // Codes q[p*ldq + c], scales sc[(c/128)*ld_s + p].
+// kPad (dispatch): E * kPadWarps further warps zero the padding rows of the
+// permuted layout, [offsets[e] + counts[e], offsets[e+1]) for each expert e,
+// codes and scales, so the padded tiles of the grouped GEMMs read zeros.
 // ---------------------------------------------------------------------------
+constexpr int kPadWarps = 8;
+
+template <bool kPad>
 __global__ void __launch_bounds__(256) quant_1x128_kernel(const uint16_t *__restrict__ in, int64_t ld,
                                                           int64_t rows, int64_t cols,
                                                           const int32_t *__restrict__ pos, int k,
                                                           uint8_t *__restrict__ q, int64_t ldq,
-                                                          float *__restrict__ sc, int64_t ld_s)
+                                                          float *__restrict__ sc, int64_t ld_s,
+                                                          const int32_t *__restrict__ counts,
+                                                          const int32_t *__restrict__ offsets, int E)
 {
     const int lane = threadIdx.x & 31;
     const int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    if (t >= rows) return;
+    if (t >= rows) {
+        if (!kPad) return;
+        const int64_t g = t - rows;
+        const int e = (int)(g / kPadWarps), w = (int)(g % kPadWarps);
+        if (e >= E) return;
+        const int64_t r1 = offsets[e + 1];
+        for (int64_t r = (int64_t)offsets[e] + counts[e] + w; r < r1; r += kPadWarps) {
+            for (int64_t c = lane * 16; c < cols; c += 512)
+                *reinterpret_cast<uint4 *>(q + r * ldq + c) = make_uint4(0, 0, 0, 0);
+            for (int64_t kb = lane; kb < cols / 128; kb += 32) sc[kb * ld_s + r] = 0.0f;
+        }
+        return;
+    }
     int my_pos = -1;
     if (pos) {
         if (lane < k) my_pos = pos[t * k + lane];
@@ -35,30 +56,40 @@ __global__ void __launch_bounds__(256) quant_1x128_kernel(const uint16_t *__rest
     }
     const int kk = pos ? k : 1;
     const uint16_t *row = in + t * ld;
-    for (int64_t c0 = 0; c0 < cols; c0 += 512) {
-        const int64_t c = c0 + lane * 16;
-        const bool act = c < cols;
-        float v[16];
-        float amax = 0.0f;
-        if (act) {
-            uint4 a = *reinterpret_cast<const uint4 *>(row + c);
-            uint4 b = *reinterpret_cast<const uint4 *>(row + c + 8);
-            unpack8(a, v);
-            unpack8(b, v + 8);
-            amax = absmax8(v + 8, absmax8(v, 0.0f));
+    for (int64_t g0 = 0; g0 < cols; g0 += 2048) {
+        uint4 buf[8];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int64_t c = g0 + 512 * u + lane * 16;
+            if (c < cols) {
+                buf[2 * u] = *reinterpret_cast<const uint4 *>(row + c);
+                buf[2 * u + 1] = *reinterpret_cast<const uint4 *>(row + c + 8);
+            } else {
+                buf[2 * u] = buf[2 * u + 1] = make_uint4(0, 0, 0, 0);
+            }
         }
-        amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
-        amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 2));
-        amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 4));
-        const float s = block_scale(amax);
-        uint4 codes = make_uint4(0, 0, 0, 0);
-        if (act) codes = quant16(v, s);
-        const int64_t kb = c / 128;
-        for (int j = 0; j < kk; ++j) {
-            int p = __shfl_sync(kFull, my_pos, j);
-            if (p >= 0 && act) {
-                *reinterpret_cast<uint4 *>(q + (int64_t)p * ldq + c) = codes;
-                if ((lane & 7) == 0) sc[kb * ld_s + p] = s;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            if (g0 + 512 * u >= cols) break;  // warp-uniform
+            const int64_t c = g0 + 512 * u + lane * 16;
+            const bool act = c < cols;
+            float v[16];
+            unpack8(buf[2 * u], v);
+            unpack8(buf[2 * u + 1], v + 8);
+            float amax = act ? absmax8(v + 8, absmax8(v, 0.0f)) : 0.0f;
+            amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
+            amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 2));
+            amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 4));
+            const float s = block_scale(amax);
+            uint4 codes = make_uint4(0, 0, 0, 0);
+            if (act) codes = quant16(v, s);
+            const int64_t kb = c / 128;
+            for (int j = 0; j < kk; ++j) {
+                const int p = __shfl_sync(kFull, my_pos, j);
+                if (p >= 0 && act) {
+                    *reinterpret_cast<uint4 *>(q + (int64_t)p * ldq + c) = codes;
+                    if ((lane & 7) == 0) sc[kb * ld_s + p] = s;
+                }
             }
         }
     }
@@ -70,7 +101,19 @@ int launch_quant_1x128(const uint16_t *in, int64_t ld, int64_t rows, int64_t col
 {
     if (rows == 0) return MOE_OK;
     int64_t blocks = (rows + 7) / 8;
-    quant_1x128_kernel<<<(unsigned)blocks, 256, 0, s>>>(in, ld, rows, cols, pos, k, q, ldq, sc, ld_s);
+    quant_1x128_kernel<false><<<(unsigned)blocks, 256, 0, s>>>(in, ld, rows, cols, pos, k, q, ldq, sc, ld_s,
+                                                               nullptr, nullptr, 0);
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int launch_dispatch_quant(const uint16_t *x, int64_t T, int64_t D, const int32_t *pos, int k, uint8_t *xq,
+                          float *xs, int64_t R_cap, const int32_t *counts, const int32_t *offsets, int E,
+                          cudaStream_t s)
+{
+    if (T == 0) return MOE_OK;  // no routed rows: every segment is empty, nothing to pad
+    const int64_t warps = T + (int64_t)E * kPadWarps;
+    quant_1x128_kernel<true><<<(unsigned)((warps + 7) / 8), 256, 0, s>>>(x, D, T, D, pos, k, xq, D, xs, R_cap,
+                                                                        counts, offsets, E);
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

@@ -74,7 +74,7 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict
 // One thread per token.  idx[t][j] = P[(layer*k + j)*T + t] (reads coalesced
 // over t).  An entry outside [0,E) or a repeated expert latches
 // MOE_ERR_BAD_ROUTING and zeroes the token's weights.
-__global__ void __launch_bounds__(256) route_replay_kernel(const int32_t *__restrict__ P, int layer,
+__global__ void __launch_bounds__(64) route_replay_kernel(const int32_t *__restrict__ P, int layer,
                                                            int T, int E, int k,
                                                            const float *__restrict__ w_in,
                                                            const float *__restrict__ z,
@@ -84,11 +84,18 @@ __global__ void __launch_bounds__(256) route_replay_kernel(const int32_t *__rest
     const int t = blockIdx.x * blockDim.x + threadIdx.x;
     if (t >= T) return;
     int e[16];
+    float wi[16];
     bool bad = false;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {  // every load first, then the checks and stores
+        if (j < k) {
+            e[j] = P[((int64_t)layer * k + j) * T + t];
+            wi[j] = w_in ? w_in[(int64_t)t * k + j] : 0.0f;
+        }
+    }
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
         if (j < k) {
-            e[j] = P[((int64_t)layer * k + j) * T + t];
             idx[(int64_t)t * k + j] = e[j];
             bad |= (e[j] < 0) || (e[j] >= E);
         }
@@ -100,11 +107,15 @@ __global__ void __launch_bounds__(256) route_replay_kernel(const int32_t *__rest
             if (jj < k) bad |= (e[j] == e[jj]);
     if (bad) {
         latch_status(status, MOE_ERR_BAD_ROUTING);
-        for (int j = 0; j < k; ++j) w[(int64_t)t * k + j] = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            if (j < k) w[(int64_t)t * k + j] = 0.0f;
         return;
     }
     if (w_in) {
-        for (int j = 0; j < k; ++j) w[(int64_t)t * k + j] = w_in[(int64_t)t * k + j];
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            if (j < k) w[(int64_t)t * k + j] = wi[j];
         return;
     }
     const float *zt = z + (int64_t)t * E;
@@ -140,7 +151,7 @@ int launch_route_replay(const int32_t *P, int layer, int T, int E, int k, const 
                         const float *z, int32_t *idx, float *w, int *status, cudaStream_t s)
 {
     if (T == 0) return MOE_OK;
-    route_replay_kernel<<<(T + 255) / 256, 256, 0, s>>>(P, layer, T, E, k, w_in, z, idx, w, status);
+    route_replay_kernel<<<(T + 63) / 64, 64, 0, s>>>(P, layer, T, E, k, w_in, z, idx, w, status);
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
