@@ -270,7 +270,7 @@ def run_ours(args, wl_name):
             abi.grouped_gemm_fp8(abi.GEMM_DOWN, d, B.offsets, B.hq, B.hs, W.wd_q, W.wd_s, out_bf16=B.Y)
             abi.combine(B.Y, B.w, B.pos, d, B.y)
 
-    launches_per_step = wl.L * (1 + 5 + 1 + 1 + 1)  # replay, permute (count/scan/place/quant/pad), 2 GEMMs, combine
+    launches_per_step = wl.L * (1 + 4 + 1 + 1 + 1)  # replay, permute (count/scan/place/dispatch quant), 2 GEMMs, combine
 
     clocks = Clocks(local, os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv")) \
         if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else Clocks(local, f"/tmp/moe_clocks_{rank}.csv")
@@ -402,6 +402,147 @@ def run_ours(args, wl_name):
     return 0
 
 
+def run_kernels(args, names):
+    """Per-stage device time of one layer pass for each named workload (the
+    stages of the hot path, forward and, for the training workload, backward):
+    each stage is captured N times in its own CUDA graph and replayed after an
+    L2 flush; the median over replays / N is its time.  Each stage reports its
+    algorithmic bytes or FLOPs (R = T*k routed rows) and the achieved fraction
+    of the measured peak (HBM copy GB/s, or 2 x bf16 burst for FP8).  One JSON
+    line per workload; not the bench line."""
+    import torch
+
+    from moe_expert_layer_replay_b200 import abi, layer
+    from moe_expert_layer_replay_b200.inputs import make_inputs
+
+    torch.cuda.set_device(0)
+    abi.lib()
+    hbm, bf16_tf, _, src = _peaks()
+    fp8 = bf16_tf * FP8_OVER_BF16
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+    for name in names:
+        inp = make_inputs(name, seed=args.seed)
+        wl = inp["workload"]
+        T, D, I, E, k = wl.T, wl.D, wl.I, wl.E, wl.k
+        R = T * k
+        d = abi.dims(T, D, I, E, k)
+        dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16) if a.dtype == np.uint16 else
+                                         np.ascontiguousarray(a)).cuda()
+        bfd = lambda a: dev(a).view(torch.bfloat16)
+        train = wl.train
+        wg, wu, wd = bfd(inp["W_gate"]), bfd(inp["W_up"]), bfd(inp["W_down"])
+        W = layer.quantise_weights(d, wg, wu, wd, train=train)
+        B = layer.Buffers(d, "cuda", train=train)
+        x = bfd(inp["x"])
+        if "payload" in inp:
+            P = dev(inp["payload"])
+            w_in = dev(inp["w_in"][0]) if "w_in" in inp else None
+            z = dev(inp["logits"]) if "logits" in inp else None
+            route = lambda: layer.route(B, payload=P, layer=0, w_in=w_in, logits=z)
+            route_bytes = 4 * R + (4 * R if w_in is not None else 4 * T * E) + 8 * R
+        else:
+            z = dev(inp["logits"])
+            route = lambda: layer.route(B, logits=z)
+            route_bytes = 4 * T * E + 8 * R
+        route()
+        abi.permute(B.idx, d, B.counts, B.offsets, B.pos, B.src, None, None, None, None, None, B.ws)
+        torch.cuda.synchronize()
+        R_pad = int(B.offsets[E].item())
+        xT = (B.xqT, B.xsT) if train else (None, None)
+        st = [
+            ("route", route, "B", route_bytes),
+            ("permute index", lambda: abi.permute(B.idx, d, B.counts, B.offsets, B.pos, B.src, None, None, None,
+                                                  None, None, B.ws), "B", 8 * R + 4 * R_pad),
+            ("permute index + dispatch quant", lambda: abi.permute(B.idx, d, B.counts, B.offsets, B.pos, B.src, x,
+                                                                   B.xq, B.xs, xT[0], xT[1], B.ws), "B",
+             8 * R + 4 * R_pad + 2 * T * D + R * (D + D // 32) + (R * (D + D // 32) if train else 0)),
+            ("gemm gate/up + SiLU + h-quant", lambda: abi.grouped_gemm_fp8(
+                abi.GEMM_GATEUP_SILU, d, B.offsets, B.xq, B.xs, W.wgu_q, W.wgu_s, aux=B.gu if train else None,
+                out_q=B.hq, out_s=B.hs, out_bf16=B.h if train else None), "F", 4.0 * R * D * I),
+            ("gemm down", lambda: abi.grouped_gemm_fp8(abi.GEMM_DOWN, d, B.offsets, B.hq, B.hs, W.wd_q, W.wd_s,
+                                                       out_bf16=B.Y), "F", 2.0 * R * D * I),
+            ("combine", lambda: abi.combine(B.Y, B.w, B.pos, d, B.y), "B", 2 * R * D + 8 * R + 2 * T * D),
+        ]
+        if train:
+            dy = bfd(inp["dy"])
+            st += [
+                ("weight quant (with transposes)", lambda: layer.quantise_weights(d, wg, wu, wd, train=True, out=W),
+                 "B", 6 * E * D * I + 2 * 3 * E * D * I * (1 + 1 / 4096)),
+                ("combine bwd", lambda: abi.combine_bwd(dy, B.Y, B.w, B.pos, B.idx, B.counts, B.offsets, d, B.dYq,
+                                                        B.dYs, B.dYb, B.d_w, B.d_logits), "B",
+                 2 * T * D + 2 * R * D + 8 * R + R * D * (1 + 1 / 32) + 2 * R * D),
+                ("128x1 quant of dY", lambda: abi.quant_fp8_block(B.dYb, B.R_cap, D, D, 128, 1, B.dYqT, B.dYsT), "B",
+                 2 * R * D + R * D * (1 + 1 / 32)),
+                ("128x1 quant of h", lambda: abi.quant_fp8_block(B.h, B.R_cap, I, I, 128, 1, B.hqT, B.hsT), "B",
+                 2 * R * I + R * I * (1 + 1 / 32)),
+                ("gemm dgrad down + SiLU bwd", lambda: abi.grouped_gemm_fp8(
+                    abi.GEMM_DGRAD_DOWN_SILU, d, B.offsets, B.dYq, B.dYs, W.wdT_q, W.wdT_s, aux=B.gu, out_q=B.dGUq,
+                    out_s=B.dGUs, out_bf16=B.dGU), "F", 2.0 * R * D * I),
+                ("128x1 quant of dGU", lambda: abi.quant_fp8_block(B.dGU, B.R_cap, 2 * I, 2 * I, 128, 1, B.dGUqT,
+                                                                   B.dGUsT), "B",
+                 4 * R * I + 2 * R * I * (1 + 1 / 32)),
+                ("gemm dgrad gate/up", lambda: abi.grouped_gemm_fp8(
+                    abi.GEMM_DGRAD_GATEUP, d, B.offsets, B.dGUq, B.dGUs, W.wguT_q, W.wguT_s, out_bf16=B.dX), "F",
+                 4.0 * R * D * I),
+                ("unpermute reduce", lambda: abi.unpermute_reduce(B.dX, B.pos, d, B.dx), "B", 2 * R * D + 2 * T * D),
+                ("gemm wgrad down", lambda: abi.grouped_gemm_fp8(abi.GEMM_WGRAD_DOWN, d, B.offsets, B.dYqT, B.dYsT,
+                                                                 B.hqT, B.hsT, out_f32=B.dWd), "F",
+                 2.0 * R * D * I),
+                ("gemm wgrad gate/up", lambda: abi.grouped_gemm_fp8(
+                    abi.GEMM_WGRAD_GATEUP, d, B.offsets, B.dGUqT, B.dGUsT, B.xqT, B.xsT, out_f32=B.dWgu), "F",
+                 4.0 * R * D * I),
+            ]
+        for _, f, _, _ in st:  # every stage once, in order (first-call set-up, valid operands)
+            f()
+        torch.cuda.synchronize()
+        if abi.get_status() != abi.OK:
+            raise RuntimeError("device status after the warm-up pass")
+        gs = torch.cuda.Stream()
+        out = []
+        for sname, f, kind, units in st:
+            n = 10 if (kind == "B" or units < 1e12) else 2
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(gs):
+                f()
+                torch.cuda.synchronize()
+                with torch.cuda.graph(g, stream=gs):
+                    for _ in range(n):
+                        f()
+            torch.cuda.synchronize()
+            ts = []
+            for r in range(max(3, args.steps // 4)):
+                flush.fill_(r & 0xFF)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                g.replay()
+                e1.record()
+                e1.synchronize()
+                ts.append(e0.elapsed_time(e1) / n)
+            del g
+            ms = statistics.median(ts)
+            if kind == "F":
+                ach = units / (ms * 1e-3) / 1e12
+                out.append({"stage": sname, "us": round(ms * 1e3, 2), "flop": units, "tflops": round(ach, 1),
+                            "frac": round(ach / fp8, 4)})
+            else:
+                ach = units / (ms * 1e-3) / 1e9
+                out.append({"stage": sname, "us": round(ms * 1e3, 2), "bytes": units, "gbs": round(ach, 1),
+                            "frac": round(ach / hbm, 4)})
+        torch.cuda.synchronize()
+        if abi.get_status() != abi.OK:
+            raise RuntimeError("device status after the timed replays")
+        gf = [o for o in out if "flop" in o]
+        line = {"kernels_report": _workload_desc(wl), "R": R, "R_pad": R_pad,
+                "peaks": {"hbm_gbs": hbm, "fp8_tflops": fp8, "source": src},
+                "gemm_tflops": round(sum(o["flop"] for o in gf) / (sum(o["us"] for o in gf) * 1e-6) / 1e12, 1),
+                "stages": out}
+        line["gemm_frac"] = round(line["gemm_tflops"] / fp8, 4)
+        print(json.dumps(line), flush=True)
+        del B, W, x
+        torch.cuda.empty_cache()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -414,7 +555,12 @@ def main():
     ap.add_argument("--ref-tokens", type=int, default=128)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch the timed steps eagerly")
+    ap.add_argument("--kernels", default=None,
+                    help="comma-separated workloads: per-stage device times and roofline fractions instead "
+                         "of the bench line")
     args = ap.parse_args()
+    if args.kernels:
+        return run_kernels(args, [w for w in args.kernels.split(",") if w])
     if args.impl == "reference":
         return run_reference(args, args.workload)
     return run_ours(args, args.workload)

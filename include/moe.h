@@ -199,8 +199,9 @@ enum {
  * DGRAD_DOWN_SILU: a = dYq [R_cap][D], sa = dYs; b = wdT_q, sb = wdT_s;
  *   aux = gu (saved by GATEUP_SILU);  dH = dY . W_down;
  *   dg = dH*u*s*(1+g*(1-s)), du = dH*silu(g), s = sigmoid(g);
- *   out_bf16 = dGU [R_cap][2I] bf16 (interleaved like wgu); out_q = dGUq
- *   [R_cap][2I] e4m3, out_s = dGUs [2I/128][R_cap] (1x128 of dGU).
+ *   out_bf16 = dGU [R_cap][2I] bf16 (interleaved like wgu; required: the
+ *   codes are made from it); out_q = dGUq [R_cap][2I] e4m3, out_s = dGUs
+ *   [2I/128][R_cap] (1x128 of dGU).
  * DGRAD_GATEUP: a = dGUq, sa = dGUs; b = wguT_q, sb = wguT_s;
  *   out_bf16 = dX [R_cap][D] bf16 (rows in permuted order).
  * WGRAD_DOWN:   a = dYqT [D][R_cap], sa = dYsT [R_cap/128][D];
@@ -209,7 +210,8 @@ enum {
  * WGRAD_GATEUP: a = dGUqT [2I][R_cap], sa = dGUsT [R_cap/128][2I];
  *               b = xqT [D][R_cap], sb = xsT [R_cap/128][D];
  *               out_f32 = dWgu [E][2I][D] fp32 (interleaved rows), +=.
- * All code/matrix pointers must be 16-byte aligned. */
+ * All code/matrix pointers must be 16-byte aligned; for the WGRAD ops the
+ * scale arrays sa and sb too. */
 typedef struct {
     const uint8_t *a;
     const float *sa;

@@ -48,14 +48,13 @@ constexpr int EPI_WARP0 = 4;
 constexpr int EPI_THREADS = 256;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint64_t DRAIN_BUDGET = 1ull << 28;
-constexpr int PF = 3;  // scale prefetch depth (K blocks)
 // smem: operand ring | barriers (full[4], empty[4], tfull[2], tempty[2], drain, epi) |
 // tmem slot | abort flag | offsets[257] | then, 1024-aligned, a region whose
 // use depends on the epilogue:
 //   SILU   amax exchange [2][2][128] fp32 | h-code store buffers [8 warps][32 rows][64 B]
 //   BF16   output store buffers [8 warps][2][32 rows][64 B]
-//   WGRAD  column-scale ring [PF][3][256] fp32 (per epilogue thread: row scale,
-//          column scale, spare)
+//   WGRAD  scale slots [STAGES][128 row + 256 column] fp32, one per operand
+//          stage, filled by the producer with the stage's tiles
 //   DSILU  unused
 // Store buffers are read by TMA stores (32 rows x 64 bytes boxes, no swizzle).
 constexpr int OFF_BAR = STAGES * STAGE_BYTES;
@@ -64,7 +63,8 @@ constexpr int OFF_ABORT = OFF_TMEM_SLOT + 4;
 constexpr int OFF_OFFSETS = OFF_BAR + 256;
 constexpr int OFF_EPI = (OFF_OFFSETS + 1040 + 1023) / 1024 * 1024;
 constexpr int OFF_AMAX = OFF_EPI;
-constexpr int OFF_RING = OFF_EPI;
+constexpr int OFF_WS = OFF_EPI;
+constexpr int WS_FLOATS = 128 + 256;
 constexpr int TSTORE_BUF = 32 * 64;
 constexpr int OFF_TSTORE_SILU = OFF_EPI + 2 * 2 * 128 * 4;
 constexpr int OFF_TSTORE_BF16 = OFF_EPI;
@@ -76,7 +76,7 @@ constexpr int smem_bytes()
 {
     return 1024 + (kEpi == EPI_SILU   ? OFF_TSTORE_SILU + 8 * TSTORE_BUF
                    : kEpi == EPI_BF16 ? OFF_TSTORE_BF16 + 8 * 2 * TSTORE_BUF
-                   : kEpi == EPI_WGRAD ? OFF_RING + PF * 3 * 256 * 4
+                   : kEpi == EPI_WGRAD ? OFF_WS + STAGES * WS_FLOATS * 4
                                        : OFF_EPI);  // + alignment slack
 }
 static_assert(smem_bytes<EPI_SILU>() <= 232448 && smem_bytes<EPI_BF16>() <= 232448 &&
@@ -179,6 +179,15 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
         " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
         : "memory");
+}
+
+// Bulk copy global -> shared (16-byte aligned, size a multiple of 16),
+// completing on an mbarrier's transaction count.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(src), "r"(bytes), "r"(bar)
+                 : "memory");
 }
 
 __device__ __forceinline__ void cp_async4(void *dst, const void *src)
@@ -332,7 +341,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_TMEM_SLOT);
     int *offs_s = reinterpret_cast<int *>(smem + OFF_OFFSETS);
     float *amax_s = reinterpret_cast<float *>(smem + OFF_AMAX);       // [2][2][128]
-    float *ring = reinterpret_cast<float *>(smem + OFF_RING);          // [PF][3][256]
+    float *wscale = reinterpret_cast<float *>(smem + OFF_WS);          // wgrad: [STAGES][WS_FLOATS]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -340,7 +349,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(bar_full + 8 * s, 1);
-            mbar_init(bar_empty + 8 * s, 1);
+            // wgrad: a stage is free again once the MMA has read its tiles and
+            // every epilogue warp has read its scales
+            mbar_init(bar_empty + 8 * s, kWgrad ? 1 + EPI_THREADS / 32 : 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(bar_tfull + 8 * b, 1);
@@ -382,11 +393,16 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     pend &= ~(1u << stage);
                     const uint32_t fb = bar_full + 8 * stage;
                     const uint32_t dA = sbase + stage * STAGE_BYTES, dB = dA + A_BYTES;
-                    mbar_arrive_expect_tx(fb, STAGE_BYTES);
                     if (kWgrad) {
+                        const int ncols = min(BN, p.N - x.n0);  // 128 or 256 (N is a multiple of 128)
+                        const uint32_t ws = smem_u32(wscale + stage * WS_FLOATS);
+                        mbar_arrive_expect_tx(fb, STAGE_BYTES + 4 * (BM + ncols));
                         tma_load_2d(dA, &tmA, kb * BK, x.m0, fb);
                         tma_load_2d(dB, &tmB, kb * BK, x.n0, fb);
+                        bulk_g2s(ws, p.sa + (int64_t)kb * p.M + x.m0, 4 * BM, fb);
+                        bulk_g2s(ws + 4 * BM, p.sb + (int64_t)kb * p.N + x.n0, 4 * ncols, fb);
                     } else {
+                        mbar_arrive_expect_tx(fb, STAGE_BYTES);
                         tma_load_2d(dA, &tmA, kb * BK, x.m0, fb);
                         tma_load_2d(dB, &tmB, kb * BK, x.e * p.N + x.n0, fb);
                     }
@@ -453,11 +469,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         const int q = warp & 3;              // TMEM lane quarter of this warp
         const int h = ew >> 2;               // column half
         const int row = 32 * q + lane;       // row within the tile
-        const int et = threadIdx.x - 32 * EPI_WARP0;  // 0..255
         const uint32_t lane_addr = tmem_base + ((uint32_t)(32 * q) << 16);
         const int KB = p.K / BK, NB = p.N / BK;
         int buf = 0;
         uint32_t bphase = 0;
+        int wstage = 0;  // wgrad: operand stage (and scale slot) of the current K block
+        uint32_t wphase = 0;
         int tcount = 0;
         bool ok = true;
         uint32_t ephase = 0;
@@ -476,8 +493,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
             // Scales of K block kb.  Rows mode: plain loads two K blocks ahead
             // into registers (row scale, weight-block scale(s)).  Wgrad: the
-            // column scales are shared by the warps, so they go through a
-            // cp.async ring in shared memory (slot kb % PF) read after a sync.
+            // producer brings them with the K block's tiles into the operand
+            // stage's scale slot; each warp releases the stage after reading.
             auto load_rows = [&](int kb, float &a, float &b0, float &b1) {
                 a = p.sa[(int64_t)kb * p.R_cap + x.m0 + row];
                 const int64_t sbrow = (int64_t)x.e * NB + 2 * x.nt;
@@ -489,36 +506,28 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     b1 = b0;
                 }
             };
-            auto issue_wgrad = [&](int kb) {
-                float *d = ring + (kb % PF) * 768;
-                cp_async4(d + et, p.sa + (int64_t)kb * p.M + x.m0 + row);
-                const int c = x.n0 + et;
-                if (c < p.N) cp_async4(d + 256 + et, p.sb + (int64_t)kb * p.N + c);
-            };
-            float c_a = 0.f, c_b0 = 0.f, c_b1 = 0.f, n_a = 0.f, n_b0 = 0.f, n_b1 = 0.f;
-            if (kWgrad) {
-                if (!epi_sync()) break;  // the previous tile's column scales are read
+            if (kEpi == EPI_DSILU && (2 * x.nt + h) * 128 < p.N) {
+                // the saved g, u this thread reads after the last K block: to L2 now
+                const uint16_t *gu = p.aux + ((int64_t)x.m0 + row) * 2 * (int64_t)p.N + (int64_t)(2 * x.nt + h) * 256;
 #pragma unroll
-                for (int j = 0; j < PF - 1; ++j) {
-                    if (x.kb0 + j < x.kb1) issue_wgrad(x.kb0 + j);
-                    cp_async_commit();
-                }
-            } else {
+                for (int j = 0; j < 4; ++j) asm volatile("prefetch.global.L2 [%0];" ::"l"(gu + 64 * j));
+            }
+            float c_a = 0.f, c_b0 = 0.f, c_b1 = 0.f, n_a = 0.f, n_b0 = 0.f, n_b1 = 0.f;
+            if (!kWgrad) {
                 load_rows(x.kb0, c_a, c_b0, c_b1);
                 if (x.kb0 + 1 < x.kb1) load_rows(x.kb0 + 1, n_a, n_b0, n_b1);
             }
             for (int kb = x.kb0; kb < x.kb1; ++kb) {
-                const float *d = ring + (kb % PF) * 768;
+                const float *d = wscale + wstage * WS_FLOATS;
                 float sa, s0, s1;
                 if (kWgrad) {
-                    cp_async_wait<PF - 2>();
-                    if (!epi_sync()) {  // everyone's column scales of kb are in
+                    // the stage's full barrier completed before the MMA of kb was
+                    // issued; waiting on it here makes the bulk-copied scales visible
+                    if (!warp_wait_bounded(bar_full + 8 * wstage, wphase, p.budget, abort_flag, p.status)) {
                         ok = false;
                         break;
                     }
-                    if (kb + PF - 1 < x.kb1) issue_wgrad(kb + PF - 1);
-                    cp_async_commit();
-                    sa = d[et];
+                    sa = d[row];
                     s0 = s1 = 0.0f;
                 } else {
                     sa = c_a;
@@ -555,7 +564,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                         }
                     }
                     if (kWgrad) {
-                        const float *cs = d + 256 + 128 * h + 32 * c;
+                        const float *cs = d + BM + 128 * h + 32 * c;
 #pragma unroll
                         for (int i = 0; i < 32; i += 2)
                             ffma2(acc[32 * c + i], acc[32 * c + i + 1], __uint_as_float(cur[i]),
@@ -568,6 +577,14 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                                   __uint_as_float(cur[i + 1]), sc, sc);
                     }
 
+                }
+                if (kWgrad) {  // this warp has read the stage's scales
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar_empty + 8 * wstage);
+                    if (++wstage == STAGES) {
+                        wstage = 0;
+                        wphase ^= 1;
+                    }
                 }
                 buf ^= 1;
                 if (buf == 0) bphase ^= 1;
@@ -643,48 +660,53 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     }
                 }
             } else if (kEpi == EPI_DSILU) {
-                // acc = dH of I-block nb = 2nt + h; gate/up columns of that block
-                // in the interleaved 2I space: 2nb*128 and (2nb+1)*128
+                // acc = dH of I-block nb = 2nt + h; its gate/up columns in the
+                // interleaved 2I space are gc = 2nb*128 and uc = gc + 128.
+                //   dg = dH u s (1 + g (1 - s)), du = dH g s, s = sigmoid(g),
+                // each rounded to bf16, stored, and quantised 1x128 (one block
+                // each).  Two passes in registers, no thread-local arrays (local
+                // memory would miss the L1 left beside this kernel's shared
+                // memory): pass 1 makes dg, du, their bf16 rows and the block
+                // maxima; pass 2 re-reads this thread's own bf16 rows (written in
+                // pass 1; the bf16 output is required for this op) and writes the
+                // codes.
                 const int nb = 2 * x.nt + h;
                 if (nb * 128 < p.N) {
                     const int64_t N2 = 2 * (int64_t)p.N;
                     const int64_t gc = (int64_t)(2 * nb) * 128, uc = gc + 128;
                     const uint16_t *gu = p.aux + r * N2;
-                    float amax_g = 0.0f, amax_u = 0.0f;
-#pragma unroll
-                    for (int i0 = 0; i0 < 128; i0 += 8) {
-                        asm volatile("" ::: "memory");  // keep one chunk's loads live at a time
-                        float g[8], u[8], dg[8], du[8];
+                    auto grads = [&](int i0, float *dg, float *du) {
+                        float g[8], u[8];
                         unpack8(*reinterpret_cast<const uint4 *>(gu + gc + i0), g);
                         unpack8(*reinterpret_cast<const uint4 *>(gu + uc + i0), u);
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
-                            const float dh = acc[i0 + i];
+                            const float d = acc[i0 + i];
                             const float sg = sigmoid_fast(g[i]);
-                            const float dgv = dh * u[i] * sg * (1.0f + g[i] * (1.0f - sg));
-                            const float duv = dh * g[i] * sg;
-                            const uint32_t bg = bf16_bits_rn(dgv), bu = bf16_bits_rn(duv);
-                            dg[i] = __uint_as_float(bg << 16);
-                            du[i] = __uint_as_float(bu << 16);
-                            amax_g = fmaxf(amax_g, fabsf(dg[i]));
-                            amax_u = fmaxf(amax_u, fabsf(du[i]));
-                            acc[i0 + i] = __uint_as_float(bg | (bu << 16));
+                            dg[i] = __uint_as_float(bf16_bits_rn(d * u[i] * sg * (1.0f + g[i] * (1.0f - sg))) << 16);
+                            du[i] = __uint_as_float(bf16_bits_rn(d * g[i] * sg) << 16);
                         }
-                        if (p.out_bf16) {
-                            *reinterpret_cast<uint4 *>(p.out_bf16 + r * N2 + gc + i0) = pack8(dg);
-                            *reinterpret_cast<uint4 *>(p.out_bf16 + r * N2 + uc + i0) = pack8(du);
-                        }
+                    };
+                    float amax_g = 0.0f, amax_u = 0.0f;
+#pragma unroll
+                    for (int i0 = 0; i0 < 128; i0 += 8) {
+                        float dg[8], du[8];
+                        grads(i0, dg, du);
+                        amax_g = absmax8(dg, amax_g);
+                        amax_u = absmax8(du, amax_u);
+                        *reinterpret_cast<uint4 *>(p.out_bf16 + r * N2 + gc + i0) = pack8(dg);
+                        *reinterpret_cast<uint4 *>(p.out_bf16 + r * N2 + uc + i0) = pack8(du);
                     }
                     const float sgs = block_scale(amax_g), sus = block_scale(amax_u);
-#pragma unroll
+                    // a rolled loop: one copy of the quantiser's code, not sixteen
+                    const uint16_t *ob = p.out_bf16 + r * N2;
+#pragma unroll 1
                     for (int i0 = 0; i0 < 128; i0 += 16) {
                         float dg[16], du[16];
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const uint32_t w = __float_as_uint(acc[i0 + i]);
-                            dg[i] = __uint_as_float(w << 16);
-                            du[i] = __uint_as_float(w & 0xffff0000u);
-                        }
+                        unpack8(*reinterpret_cast<const uint4 *>(ob + gc + i0), dg);
+                        unpack8(*reinterpret_cast<const uint4 *>(ob + gc + i0 + 8), dg + 8);
+                        unpack8(*reinterpret_cast<const uint4 *>(ob + uc + i0), du);
+                        unpack8(*reinterpret_cast<const uint4 *>(ob + uc + i0 + 8), du + 8);
                         *reinterpret_cast<uint4 *>(p.out_q + r * N2 + gc + i0) = quant16(dg, sgs);
                         *reinterpret_cast<uint4 *>(p.out_q + r * N2 + uc + i0) = quant16(du, sus);
                     }

@@ -216,12 +216,14 @@ int moe_grouped_gemm_fp8(int32_t op, const moe_dims *d, const int32_t *offsets, 
         if (!g->out_bf16 || !aligned16(g->out_bf16)) return MOE_ERR_INVALID_ARG;
         break;
     case MOE_GEMM_DGRAD_DOWN_SILU:
-        if (!g->aux || !g->out_q || !g->out_s || !aligned16(g->aux) || !aligned16(g->out_q)) return MOE_ERR_INVALID_ARG;
-        if (g->out_bf16 && !aligned16(g->out_bf16)) return MOE_ERR_INVALID_ARG;
+        if (!g->aux || !g->out_q || !g->out_s || !g->out_bf16 || !aligned16(g->aux) || !aligned16(g->out_q) ||
+            !aligned16(g->out_bf16))
+            return MOE_ERR_INVALID_ARG;
         break;
     case MOE_GEMM_WGRAD_DOWN:
-    case MOE_GEMM_WGRAD_GATEUP:
-        if (!g->out_f32 || !aligned16(g->out_f32)) return MOE_ERR_INVALID_ARG;
+    case MOE_GEMM_WGRAD_GATEUP:  // the scale rows are bulk-copied: 16-byte alignment
+        if (!g->out_f32 || !aligned16(g->out_f32) || !aligned16(g->sa) || !aligned16(g->sb))
+            return MOE_ERR_INVALID_ARG;
         break;
     default:
         return MOE_ERR_INVALID_ARG;
