@@ -564,11 +564,17 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                         }
                     }
                     if (kWgrad) {
-                        const float *cs = d + BM + 128 * h + 32 * c;
+                        // column scales of this chunk: 16-byte shared loads (a slot is
+                        // 1536 B, the column part starts 512 B in)
+                        const float4 *cs = reinterpret_cast<const float4 *>(d + BM + 128 * h + 32 * c);
 #pragma unroll
-                        for (int i = 0; i < 32; i += 2)
+                        for (int i = 0; i < 32; i += 4) {
+                            const float4 c4 = cs[i >> 2];
                             ffma2(acc[32 * c + i], acc[32 * c + i + 1], __uint_as_float(cur[i]),
-                                  __uint_as_float(cur[i + 1]), sa * cs[i], sa * cs[i + 1]);
+                                  __uint_as_float(cur[i + 1]), sa * c4.x, sa * c4.y);
+                            ffma2(acc[32 * c + i + 2], acc[32 * c + i + 3], __uint_as_float(cur[i + 2]),
+                                  __uint_as_float(cur[i + 3]), sa * c4.z, sa * c4.w);
+                        }
                     } else {
                         const float sc = (kEpi == EPI_SILU && c >= 2) ? s1 : s0;
 #pragma unroll

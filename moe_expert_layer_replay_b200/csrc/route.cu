@@ -71,6 +71,65 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict
     }
 }
 
+// E <= 32: one thread per token with its E logits in registers (16-byte
+// loads when E is a multiple of 4); each of the k rounds scans them in index
+// order for the best untaken (value desc, index asc), as the warp form does.
+__global__ void __launch_bounds__(128) route_topk_small_kernel(const float *__restrict__ z, int T, int E,
+                                                               int k, int32_t *__restrict__ idx,
+                                                               float *__restrict__ w)
+{
+    const int t = blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= T) return;
+    const float *zt = z + (int64_t)t * E;
+    float v[32];
+    if ((E & 3) == 0 && (reinterpret_cast<uintptr_t>(z) & 15u) == 0) {
+#pragma unroll
+        for (int e4 = 0; e4 < 32; e4 += 4) {
+            float4 q = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+            if (e4 < E) q = *reinterpret_cast<const float4 *>(zt + e4);
+            v[e4] = q.x, v[e4 + 1] = q.y, v[e4 + 2] = q.z, v[e4 + 3] = q.w;
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] = (e < E) ? zt[e] : -INFINITY;
+    }
+    uint32_t taken = (E < 32) ? ~((1u << E) - 1u) : 0u;
+    float sv[16];
+    int se[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        sv[j] = -INFINITY;
+        se[j] = 0;
+        if (j < k) {
+            float bv = -INFINITY;
+            int be = 0x7fffffff;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                if (!((taken >> e) & 1u) && (v[e] > bv || (v[e] == bv && e < be))) {
+                    bv = v[e];
+                    be = e;
+                }
+            }
+            taken |= 1u << (be & 31);
+            sv[j] = bv;
+            se[j] = be;
+        }
+    }
+    // softmax over the chosen set; round 0 holds the largest logit
+    float ex[16], sum = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        ex[j] = (j < k) ? expf(sv[j] - sv[0]) : 0.0f;
+        sum += ex[j];
+    }
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+        if (j < k) {
+            idx[(int64_t)t * k + j] = se[j];
+            w[(int64_t)t * k + j] = ex[j] / sum;
+        }
+}
+
 // One thread per token.  idx[t][j] = P[(layer*k + j)*T + t] (reads coalesced
 // over t).  An entry outside [0,E) or a repeated expert latches
 // MOE_ERR_BAD_ROUTING and zeroes the token's weights.
@@ -142,8 +201,12 @@ __global__ void __launch_bounds__(64) route_replay_kernel(const int32_t *__restr
 int launch_route_topk(const float *z, int T, int E, int k, int32_t *idx, float *w, cudaStream_t s)
 {
     if (T == 0) return MOE_OK;
-    int blocks = (T + 7) / 8;
-    route_topk_kernel<<<blocks, 256, 0, s>>>(z, T, E, k, idx, w);
+    if (E <= 32) {
+        route_topk_small_kernel<<<(T + 127) / 128, 128, 0, s>>>(z, T, E, k, idx, w);
+    } else {
+        const int blocks = (T + 7) / 8;
+        route_topk_kernel<<<blocks, 256, 0, s>>>(z, T, E, k, idx, w);
+    }
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
