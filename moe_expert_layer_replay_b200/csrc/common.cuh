@@ -69,25 +69,28 @@ __device__ __forceinline__ float block_scale(float amax) { return __fdiv_rn(amax
 // without a divide per element and without a branch.
 //
 // With r = RN(1/s), q' = RN(x * r) = (x/s)(1 + d), |d| < 3 * 2^-24, so q' is
-// within 3 fp32 ulps of q.  e4m3 (3 mantissa bits) rounds q and q' to
-// different codes only if an e4m3 rounding midpoint M lies between them or on
-// one of them.  In e4m3's normal range a midpoint is an fp32 value whose 20
-// low mantissa bits are 0x80000; q' is "near" when those bits are within 4 of
-// it.  Below 2^-6 (e4m3's subnormal grid, step 2^-9) the midpoints are the
-// odd multiples of 2^-10; adding 2^-6 maps them onto the midpoints of the
-// binade [2^-6, 2^-5) (same step), where the same bit test applies (the
-// addition's rounding adds at most half an ulp of the window).
+// within 3 fp32 ulps of q.  Let M be the e4m3 rounding midpoint of the bracket
+// [V_j, V_j+1) of e4m3 values that holds q'.  In e4m3's normal range M has
+// q''s sign, exponent and top three mantissa bits, then a 1 (20 low mantissa
+// bits 0x80000).  Below 2^-6 (e4m3's subnormal grid, step 2^-9) the midpoints
+// are the odd multiples of 2^-10: adding 2^-6 with rounding toward zero maps
+// q' into [2^-6, 2^-5), whose brackets are the same 2^-9 steps (the boundaries
+// are representable, so the truncated sum lies in the exact sum's bracket).
 //
-// A near element is decided exactly against M: q > M iff x/s > M + u/2,
-// q < M iff x/s < M - u/2, else q == M (u = fp32 ulp of M; M has 4 significant
-// bits, so its last fp32 mantissa bit is 0 and ties at M +- u/2 round to M;
-// the one midpoint that is a power of two, 2^-10, ties down to the code 0
-// either way).  For a near element x - M*s is a small multiple of the grid of
-// M*s (at most 11 significant bits), so fma(-M, s, |x|) is that difference
-// exactly, and it is compared with the exact u/2 * s.  This needs
-// s >= 2^-100 (no underflow in the grid or in u/2 * s); smaller scales take
-// the IEEE division.  The element converts through M, or its fp32 neighbour
-// on the decided side, which e4m3 rounds like q.
+// q rounds like M's neighbours: q > M iff x/s > M + u/2, q < M iff x/s <
+// M - u/2, else q == M (u = fp32 ulp of M; M has 4 significant bits, so its
+// last fp32 mantissa bit is 0 and ties at M +- u/2 round to M; the one
+// midpoint that is a power of two, 2^-10, ties down to code 0 either way).
+// The test compares e = fma(-M, s, |x|) with c = s * u/2 (exact: a power-of-two
+// multiple of s):
+//   - when q' is within 4 ulps of M, x - M*s is a small multiple of the grid
+//     of M*s (at most 11 significant bits), so e is that difference exactly;
+//   - otherwise |x/s - M| > 1 ulp of M (1.5 * 2^-29 below 2^-6), so |x - M*s|
+//     > 2c and the rounded e falls on the same side of +-c as the exact one.
+// The element then converts through M or its fp32 neighbour on the decided
+// side, which e4m3 rounds like q.  Scales below 2^-90 use IEEE division:
+// from there up, c (>= s * 2^-34) and the grid of M*s (>= 2^-126 for M >=
+// 2^-10) stay in fp32's normal range, so neither is rounded.
 template <int n>
 struct Floats {
     float v[n];
@@ -107,7 +110,7 @@ template <int n>
 __device__ __forceinline__ void quotients(const float *v, float s, float *q)
 {
     const float r = __frcp_rn(s);
-    if (!(r <= 0x1p100f)) {  // s below about 2^-100: IEEE division, out of line
+    if (!(r <= 0x1p90f)) {  // s below about 2^-90: IEEE division, out of line
         Floats<n> x;
 #pragma unroll
         for (int i = 0; i < n; ++i) x.v[i] = v[i];
@@ -122,14 +125,13 @@ __device__ __forceinline__ void quotients(const float *v, float s, float *q)
         const float qp = __fmul_rn(v[i], r);
         const uint32_t b = __float_as_uint(qp) & 0x7fffffffu;
         const bool sub = b < 0x3c800000u;
-        const uint32_t y = sub ? __float_as_uint(__fadd_rn(__uint_as_float(b), 0x1p-6f)) : b;
-        const bool near = ((y - 0x7fffcu) & 0xfffffu) <= 8u;
+        const uint32_t y = sub ? __float_as_uint(__fadd_rz(__uint_as_float(b), 0x1p-6f)) : b;
         const float My = __uint_as_float((y & 0xfff00000u) | 0x00080000u);
         const float M = sub ? __fsub_rn(My, 0x1p-6f) : My;
         const float c = __fmul_rn(s24, __uint_as_float(__float_as_uint(M) & 0x7f800000u));
         const float e = __fmaf_rn(-M, s, fabsf(v[i]));
         const uint32_t mb = __float_as_uint(M) + (e > c ? 1u : 0u) - (e < -c ? 1u : 0u);
-        q[i] = near ? __uint_as_float(mb | (__float_as_uint(qp) & 0x80000000u)) : qp;
+        q[i] = __uint_as_float(mb | (__float_as_uint(qp) & 0x80000000u));
     }
 }
 
