@@ -105,35 +105,52 @@ __global__ void __launch_bounds__(256) combine_bwd_kernel(
             for (int i = 0; i < 16; ++i) g[i] = 0.0f;
         }
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            if (j >= k) break;
-            const int p = __shfl_sync(kFull, my_pos, j);
-            const float wj = __shfl_sync(kFull, my_w, j);
-            float v[16];
-            float amax = 0.0f;
+        for (int j0 = 0; j0 < 16; j0 += 4) {
+            if (j0 >= k) break;
+            // the Y rows of up to 4 slots are loaded before any is used
+            uint4 yr[4][2];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                // the product in fp32, then bf16: the rounding point of a dY row
-                float prod = __fmul_rn(wj, g[i]);
-                v[i] = __uint_as_float(bf16_bits_rn(prod) << 16);
-                amax = fmaxf(amax, fabsf(v[i]));
-            }
-            amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
-            amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 2));
-            amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 4));
-            const float s = block_scale(amax);
-            if (act && p >= 0) {
-                *reinterpret_cast<uint4 *>(dYq + (int64_t)p * D + c) = quant16(v, s);
-                if ((lane & 7) == 0) dYs[(int64_t)(c / 128) * R_cap + p] = s;
-                if (dYb) {
-                    *reinterpret_cast<uint4 *>(dYb + (int64_t)p * D + c) = pack8(v);
-                    *reinterpret_cast<uint4 *>(dYb + (int64_t)p * D + c + 8) = pack8(v + 8);
+            for (int u = 0; u < 4; ++u) {
+                const int j = j0 + u;
+                const int p = __shfl_sync(kFull, my_pos, j & 31);
+                yr[u][0] = yr[u][1] = make_uint4(0, 0, 0, 0);
+                if (act && j < k && p >= 0) {
+                    yr[u][0] = *reinterpret_cast<const uint4 *>(Y + (int64_t)p * D + c);
+                    yr[u][1] = *reinterpret_cast<const uint4 *>(Y + (int64_t)p * D + c + 8);
                 }
-                float yv[16];
-                unpack8(*reinterpret_cast<const uint4 *>(Y + (int64_t)p * D + c), yv);
-                unpack8(*reinterpret_cast<const uint4 *>(Y + (int64_t)p * D + c + 8), yv + 8);
+            }
 #pragma unroll
-                for (int i = 0; i < 16; ++i) dw_part[j] = fmaf(g[i], yv[i], dw_part[j]);
+            for (int u = 0; u < 4; ++u) {
+                const int j = j0 + u;
+                if (j >= k) break;
+                const int p = __shfl_sync(kFull, my_pos, j);
+                const float wj = __shfl_sync(kFull, my_w, j);
+                float v[16];
+                float amax = 0.0f;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    // the product in fp32, then bf16: the rounding point of a dY row
+                    float prod = __fmul_rn(wj, g[i]);
+                    v[i] = __uint_as_float(bf16_bits_rn(prod) << 16);
+                    amax = fmaxf(amax, fabsf(v[i]));
+                }
+                amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
+                amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 2));
+                amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 4));
+                const float s = block_scale(amax);
+                if (act && p >= 0) {
+                    *reinterpret_cast<uint4 *>(dYq + (int64_t)p * D + c) = quant16(v, s);
+                    if ((lane & 7) == 0) dYs[(int64_t)(c / 128) * R_cap + p] = s;
+                    if (dYb) {
+                        *reinterpret_cast<uint4 *>(dYb + (int64_t)p * D + c) = pack8(v);
+                        *reinterpret_cast<uint4 *>(dYb + (int64_t)p * D + c + 8) = pack8(v + 8);
+                    }
+                    float yv[16];
+                    unpack8(yr[u][0], yv);
+                    unpack8(yr[u][1], yv + 8);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) dw_part[j] = fmaf(g[i], yv[i], dw_part[j]);
+                }
             }
         }
     }

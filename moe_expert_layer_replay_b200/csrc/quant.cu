@@ -132,7 +132,9 @@ __global__ void __launch_bounds__(256) quant_rows128_kernel(const uint16_t *__re
                                                             uint8_t *__restrict__ qT,
                                                             float *__restrict__ sT)
 {
-    __shared__ float tile[128][65];
+    // bf16 tile, rows of 64 columns + 8 pad (144 B: 16-byte aligned rows, and a
+    // warp's 32 consecutive columns of one row are 64 contiguous bytes)
+    __shared__ __align__(16) uint16_t tile[128][72];
     __shared__ float part_max[4][64];
     const int tid = threadIdx.x;
     const int64_t r0 = (int64_t)blockIdx.x * 128;
@@ -151,34 +153,29 @@ __global__ void __launch_bounds__(256) quant_rows128_kernel(const uint16_t *__re
                 src = in + gr * ld;
             }
         }
-        float v[8];
-        if (src && c0 + cc < cols) {
-            unpack8(*reinterpret_cast<const uint4 *>(src + c0 + cc), v);
-        } else {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) v[i] = 0.0f;
-        }
-#pragma unroll
-        for (int i = 0; i < 8; ++i) tile[r][cc + i] = v[i];
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (src && c0 + cc < cols) v = *reinterpret_cast<const uint4 *>(src + c0 + cc);
+        *reinterpret_cast<uint4 *>(&tile[r][cc]) = v;
     }
     __syncthreads();
     const int col = tid & 63, part = tid >> 6;
+    float v[32];  // this thread's 32 rows of its column
     float amax = 0.0f;
-#pragma unroll 8
-    for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(tile[part * 32 + i][col]));
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        v[i] = __uint_as_float((uint32_t)tile[part * 32 + i][col] << 16);
+        amax = fmaxf(amax, fabsf(v[i]));
+    }
     part_max[part][col] = amax;
     __syncthreads();
     amax = fmaxf(fmaxf(part_max[0][col], part_max[1][col]), fmaxf(part_max[2][col], part_max[3][col]));
     const float s = block_scale(amax);
     const int64_t gc = c0 + col;
     if (gc >= cols) return;
-    float v[16];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-        int64_t rr = r0 + part * 32 + h * 16;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = tile[part * 32 + h * 16 + i][col];
-        uint4 codes = quant16(v, s);
+        const int64_t rr = r0 + part * 32 + h * 16;
+        const uint4 codes = quant16(v + 16 * h, s);
         if (rr < rows) *reinterpret_cast<uint4 *>(qT + gc * ld_rows + rr) = codes;
     }
     if (part == 0) sT[(r0 / 128) * cols + gc] = s;
