@@ -286,12 +286,13 @@ __global__ void __launch_bounds__(256) quant_128x128_kernel(
     if (!qT) return;
     __syncthreads();
     // transposed: tile column c -> 128 bytes of qT row (cb*128 + c); each
-    // thread assembles 16 codes (rows 16*h .. 16*h+15) of one column
+    // thread assembles 16 codes (rows 16*h .. 16*h+15) of one column.  A warp
+    // takes 32 consecutive columns of the same rows (no shared-memory bank
+    // conflicts: the rows 16 apart of one column would share a bank).
     uint8_t *qTe = qT + e * qT_es;
 #pragma unroll
     for (int it = 0; it < 4; ++it) {
-        int piece = it * 256 + tid;  // 128 columns x 8 pieces
-        int c = piece >> 3, h = piece & 7;
+        const int c = tid & 127, h = 2 * it + (tid >> 7);  // 128 columns x 8 pieces
         uint32_t w[4];
 #pragma unroll
         for (int b = 0; b < 4; ++b) {
