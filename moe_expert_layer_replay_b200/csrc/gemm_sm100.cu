@@ -53,8 +53,9 @@ constexpr uint64_t DRAIN_BUDGET = 1ull << 28;
 // use depends on the epilogue:
 //   SILU   amax exchange [2][2][128] fp32 | h-code store buffers [8 warps][32 rows][64 B]
 //   BF16   output store buffers [8 warps][2][32 rows][64 B]
-//   WGRAD  scale slots [STAGES][128 row + 256 column] fp32, one per operand
-//          stage, filled by the producer with the stage's tiles
+//   WGRAD  scale ring [SC_SLOTS][128 row + 256 column] fp32 with its own
+//          full/empty barriers (filled by the producer, released by the
+//          epilogue warps), deeper than the operand ring
 //   DSILU  unused
 // Store buffers are read by TMA stores (32 rows x 64 bytes boxes, no swizzle).
 constexpr int OFF_BAR = STAGES * STAGE_BYTES;
@@ -65,6 +66,8 @@ constexpr int OFF_EPI = (OFF_OFFSETS + 1040 + 1023) / 1024 * 1024;
 constexpr int OFF_AMAX = OFF_EPI;
 constexpr int OFF_WS = OFF_EPI;
 constexpr int WS_FLOATS = 128 + 256;
+constexpr int SC_SLOTS = 8;
+constexpr int OFF_WS_BAR = OFF_WS + SC_SLOTS * WS_FLOATS * 4;  // sfull[SC_SLOTS], sempty[SC_SLOTS]
 constexpr int TSTORE_BUF = 32 * 64;
 constexpr int OFF_TSTORE_SILU = OFF_EPI + 2 * 2 * 128 * 4;
 constexpr int OFF_TSTORE_BF16 = OFF_EPI;
@@ -76,7 +79,7 @@ constexpr int smem_bytes()
 {
     return 1024 + (kEpi == EPI_SILU   ? OFF_TSTORE_SILU + 8 * TSTORE_BUF
                    : kEpi == EPI_BF16 ? OFF_TSTORE_BF16 + 8 * 2 * TSTORE_BUF
-                   : kEpi == EPI_WGRAD ? OFF_WS + STAGES * WS_FLOATS * 4
+                   : kEpi == EPI_WGRAD ? OFF_WS_BAR + 2 * SC_SLOTS * 8
                                        : OFF_EPI);  // + alignment slack
 }
 static_assert(smem_bytes<EPI_SILU>() <= 232448 && smem_bytes<EPI_BF16>() <= 232448 &&
@@ -341,7 +344,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_TMEM_SLOT);
     int *offs_s = reinterpret_cast<int *>(smem + OFF_OFFSETS);
     float *amax_s = reinterpret_cast<float *>(smem + OFF_AMAX);       // [2][2][128]
-    float *wscale = reinterpret_cast<float *>(smem + OFF_WS);          // wgrad: [STAGES][WS_FLOATS]
+    float *wscale = reinterpret_cast<float *>(smem + OFF_WS);          // wgrad: [SC_SLOTS][WS_FLOATS]
+    const uint32_t bar_sfull = sbase + OFF_WS_BAR;                     // wgrad: [SC_SLOTS]
+    const uint32_t bar_sempty = bar_sfull + SC_SLOTS * 8;              // wgrad: [SC_SLOTS]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -349,10 +354,13 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(bar_full + 8 * s, 1);
-            // wgrad: a stage is free again once the MMA has read its tiles and
-            // every epilogue warp has read its scales
-            mbar_init(bar_empty + 8 * s, kWgrad ? 1 + EPI_THREADS / 32 : 1);
+            mbar_init(bar_empty + 8 * s, 1);
         }
+        if (kWgrad)
+            for (int s = 0; s < SC_SLOTS; ++s) {
+                mbar_init(bar_sfull + 8 * s, 1);
+                mbar_init(bar_sempty + 8 * s, EPI_THREADS / 32);
+            }
         for (int b = 0; b < 2; ++b) {
             mbar_init(bar_tfull + 8 * b, 1);
             mbar_init(bar_tempty + 8 * b, EPI_THREADS / 32);
@@ -382,6 +390,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             int stage = 0;
             uint32_t phase = 0;
             uint32_t pend = 0, pend_phase = 0;  // loads issued, not yet seen consumed
+            int sslot = 0;                      // wgrad scale ring
+            uint32_t sphase = 0, spend = 0, spend_phase = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
                 const Tile x = tile_of<kWgrad>(t, p, offs_s);
@@ -394,13 +404,26 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     const uint32_t fb = bar_full + 8 * stage;
                     const uint32_t dA = sbase + stage * STAGE_BYTES, dB = dA + A_BYTES;
                     if (kWgrad) {
+                        // the K block's scales into the next slot of the scale ring
+                        if (!wait_bounded(bar_sempty + 8 * sslot, sphase ^ 1, p.budget, abort_flag, p.status)) {
+                            ok = false;
+                            break;
+                        }
+                        spend &= ~(1u << sslot);
                         const int ncols = min(BN, p.N - x.n0);  // 128 or 256 (N is a multiple of 128)
-                        const uint32_t ws = smem_u32(wscale + stage * WS_FLOATS);
-                        mbar_arrive_expect_tx(fb, STAGE_BYTES + 4 * (BM + ncols));
+                        const uint32_t ws = smem_u32(wscale + sslot * WS_FLOATS), sfb = bar_sfull + 8 * sslot;
+                        mbar_arrive_expect_tx(sfb, 4 * (BM + ncols));
+                        bulk_g2s(ws, p.sa + (int64_t)kb * p.M + x.m0, 4 * BM, sfb);
+                        bulk_g2s(ws + 4 * BM, p.sb + (int64_t)kb * p.N + x.n0, 4 * ncols, sfb);
+                        spend |= 1u << sslot;
+                        spend_phase = (spend_phase & ~(1u << sslot)) | (sphase << sslot);
+                        if (++sslot == SC_SLOTS) {
+                            sslot = 0;
+                            sphase ^= 1;
+                        }
+                        mbar_arrive_expect_tx(fb, STAGE_BYTES);
                         tma_load_2d(dA, &tmA, kb * BK, x.m0, fb);
                         tma_load_2d(dB, &tmB, kb * BK, x.n0, fb);
-                        bulk_g2s(ws, p.sa + (int64_t)kb * p.M + x.m0, 4 * BM, fb);
-                        bulk_g2s(ws + 4 * BM, p.sb + (int64_t)kb * p.N + x.n0, 4 * ncols, fb);
                     } else {
                         mbar_arrive_expect_tx(fb, STAGE_BYTES);
                         tma_load_2d(dA, &tmA, kb * BK, x.m0, fb);
@@ -417,6 +440,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             if (!ok) {
                 for (int s = 0; s < STAGES; ++s)
                     if (pend & (1u << s)) wait_drain(bar_full + 8 * s, (pend_phase >> s) & 1u);
+                if (kWgrad)
+                    for (int s = 0; s < SC_SLOTS; ++s)
+                        if (spend & (1u << s)) wait_drain(bar_sfull + 8 * s, (spend_phase >> s) & 1u);
             }
         }
     } else if (warp == 1) {
@@ -473,7 +499,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         const int KB = p.K / BK, NB = p.N / BK;
         int buf = 0;
         uint32_t bphase = 0;
-        int wstage = 0;  // wgrad: operand stage (and scale slot) of the current K block
+        int wstage = 0;  // wgrad: scale-ring slot of the current K block
         uint32_t wphase = 0;
         int tcount = 0;
         bool ok = true;
@@ -493,8 +519,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
             // Scales of K block kb.  Rows mode: plain loads two K blocks ahead
             // into registers (row scale, weight-block scale(s)).  Wgrad: the
-            // producer brings them with the K block's tiles into the operand
-            // stage's scale slot; each warp releases the stage after reading.
+            // producer bulk-copies them into the scale ring, up to SC_SLOTS K
+            // blocks ahead; each warp releases a slot after reading it.
             auto load_rows = [&](int kb, float &a, float &b0, float &b1) {
                 a = p.sa[(int64_t)kb * p.R_cap + x.m0 + row];
                 const int64_t sbrow = (int64_t)x.e * NB + 2 * x.nt;
@@ -521,9 +547,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 const float *d = wscale + wstage * WS_FLOATS;
                 float sa, s0, s1;
                 if (kWgrad) {
-                    // the stage's full barrier completed before the MMA of kb was
-                    // issued; waiting on it here makes the bulk-copied scales visible
-                    if (!warp_wait_bounded(bar_full + 8 * wstage, wphase, p.budget, abort_flag, p.status)) {
+                    if (!warp_wait_bounded(bar_sfull + 8 * wstage, wphase, p.budget, abort_flag, p.status)) {
                         ok = false;
                         break;
                     }
@@ -584,10 +608,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     }
 
                 }
-                if (kWgrad) {  // this warp has read the stage's scales
+                if (kWgrad) {  // this warp has read the slot's scales
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(bar_empty + 8 * wstage);
-                    if (++wstage == STAGES) {
+                    if (lane == 0) mbar_arrive(bar_sempty + 8 * wstage);
+                    if (++wstage == SC_SLOTS) {
                         wstage = 0;
                         wphase ^= 1;
                     }
