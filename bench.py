@@ -42,7 +42,7 @@ FP8_OVER_BF16 = 2.0  # nominal dense ratio (4.5 / 2.25 PFLOP/s)
 # workload, from the ncu capture summarised in profiles/grouped_gemm_replay_ncu.md.
 # Valid only for the kernel sources it was taken on: reported as null as soon
 # as their hash differs.
-GEMM1_TRAFFIC = {"sources_sha256_16": "442a7ecc3c468813", "bytes": 356.301312e6}
+GEMM1_TRAFFIC = {"sources_sha256_16": "898c98b641d524a5", "bytes": 360.218624e6}
 
 
 def _gemm_sources_hash() -> str:
