@@ -83,24 +83,73 @@ __global__ void __launch_bounds__(256) perm_scan_kernel(const int32_t *__restric
     }
 }
 
+// kFused (few blocks): the scan pass is done here, by every block for itself:
+// per expert the total over all blocks' counts and this block's base, then
+// the padded offsets (block 0 stores counts and offsets).  Otherwise counts,
+// offsets and bases come from perm_scan_kernel.
+template <bool kFused>
 __global__ void __launch_bounds__(256) perm_place_kernel(const int32_t *__restrict__ idx, int64_t n,
-                                                         int E, const int32_t *__restrict__ blkbase,
-                                                         const int32_t *__restrict__ offsets,
-                                                         const int32_t *__restrict__ counts, int64_t R_cap,
+                                                         int E, int align, int nblk,
+                                                         const int32_t *__restrict__ blkcnt,
+                                                         const int32_t *__restrict__ blkbase,
+                                                         int32_t *__restrict__ offsets,
+                                                         int32_t *__restrict__ counts, int64_t R_cap,
                                                          int32_t *__restrict__ pos,
                                                          int32_t *__restrict__ src_idx, int *status)
 {
+    __shared__ int s_off[257], s_cnt[256], s_base[256];
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    if (kFused) {
+        for (int e = threadIdx.x; e < E; e += blockDim.x) {
+            int tot = 0, base = 0;
+            for (int b = 0; b < nblk; ++b) {
+                const int c = blkcnt[(int64_t)b * E + e];
+                if (b < (int)blockIdx.x) base += c;
+                tot += c;
+            }
+            s_cnt[e] = tot;
+            s_base[e] = base;
+        }
+        __syncthreads();
+        if (wid == 0) {  // exclusive scan of the padded sizes, 32 experts per step
+            int carry = 0;
+            for (int e0 = 0; e0 < E; e0 += 32) {
+                const int e = e0 + lane;
+                const int v = e < E ? (s_cnt[e] + align - 1) / align * align : 0;
+                int x = v;
+#pragma unroll
+                for (int d = 1; d < 32; d <<= 1) {
+                    const int y = __shfl_up_sync(kFull, x, d);
+                    if (lane >= d) x += y;
+                }
+                if (e < E) s_off[e] = carry + x - v;
+                carry += __shfl_sync(kFull, x, 31);
+            }
+            if (lane == 0) s_off[E] = carry;
+        }
+        __syncthreads();
+        if (blockIdx.x == 0) {
+            for (int e = threadIdx.x; e < E; e += blockDim.x) counts[e] = s_cnt[e];
+            for (int e = threadIdx.x; e <= E; e += blockDim.x) offsets[e] = s_off[e];
+        }
+    } else {
+        for (int e = threadIdx.x; e < E; e += blockDim.x) {
+            s_cnt[e] = counts[e];
+            s_base[e] = blkbase[(int64_t)blockIdx.x * E + e];
+        }
+        for (int e = threadIdx.x; e <= E; e += blockDim.x) s_off[e] = offsets[e];
+        __syncthreads();
+    }
     // rows no entry fills: expert e's padding goes to block e % gridDim.x;
     // the rows past offsets[E] are shared by all blocks
     for (int e = blockIdx.x; e < E; e += gridDim.x)
-        for (int64_t r = (int64_t)offsets[e] + counts[e] + threadIdx.x; r < offsets[e + 1]; r += blockDim.x)
+        for (int64_t r = (int64_t)s_off[e] + s_cnt[e] + threadIdx.x; r < s_off[e + 1]; r += blockDim.x)
             src_idx[r] = -1;
-    for (int64_t r = (int64_t)offsets[E] + (int64_t)blockIdx.x * blockDim.x + threadIdx.x; r < R_cap;
+    for (int64_t r = (int64_t)s_off[E] + (int64_t)blockIdx.x * blockDim.x + threadIdx.x; r < R_cap;
          r += (int64_t)gridDim.x * blockDim.x)
         src_idx[r] = -1;
     if (n == 0) return;
     extern __shared__ int whist[];  // [kPlaceWarps][E]
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     for (int i = threadIdx.x; i < kPlaceWarps * E; i += blockDim.x) whist[i] = 0;
     __syncthreads();
     constexpr int sub = kChunk / kPlaceWarps;
@@ -114,7 +163,7 @@ __global__ void __launch_bounds__(256) perm_place_kernel(const int32_t *__restri
     }
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        int run = offsets[e] + blkbase[(int64_t)blockIdx.x * E + e];
+        int run = s_off[e] + s_base[e];
         for (int w = 0; w < kPlaceWarps; ++w) {
             int c = whist[w * E + e];
             whist[w * E + e] = run;
@@ -154,10 +203,18 @@ int launch_permute_index(const int32_t *idx, int T, int k, int E, int align, int
     if (nblk > 0) {
         perm_count_kernel<<<nblk, 256, E * sizeof(int), s>>>(idx, n, E, blkcnt);
     }
-    perm_scan_kernel<<<1, 256, 0, s>>>(blkcnt, nblk, E, align, blkbase, counts, offsets);
-    // place also writes -1 to the rows of src_idx that no entry fills
-    perm_place_kernel<<<nblk > 0 ? nblk : 1, 32 * kPlaceWarps, kPlaceWarps * E * sizeof(int), s>>>(
-        idx, n, E, blkbase, offsets, counts, R_cap, pos, src_idx, status);
+    // place also writes -1 to the rows of src_idx that no entry fills; with
+    // few blocks it does the scan pass itself (one launch less)
+    const int pblk = nblk > 0 ? nblk : 1;
+    const size_t psmem = kPlaceWarps * E * sizeof(int);
+    if (nblk <= 64) {
+        perm_place_kernel<true><<<pblk, 32 * kPlaceWarps, psmem, s>>>(idx, n, E, align, nblk, blkcnt, blkbase,
+                                                                     offsets, counts, R_cap, pos, src_idx, status);
+    } else {
+        perm_scan_kernel<<<1, 256, 0, s>>>(blkcnt, nblk, E, align, blkbase, counts, offsets);
+        perm_place_kernel<false><<<pblk, 32 * kPlaceWarps, psmem, s>>>(idx, n, E, align, nblk, blkcnt, blkbase,
+                                                                      offsets, counts, R_cap, pos, src_idx, status);
+    }
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
