@@ -39,3 +39,28 @@ def test_host_only_calls():
                                           ctypes.byref(g), None) == abi.UNSUPPORTED
     assert abi.lib().moe_grouped_gemm_fp8(0, ctypes.byref(abi.dims(16, 256, 128, 8, 2)), None,
                                           ctypes.byref(g), None) == abi.INVALID_ARG
+
+
+def test_gemm_operand_contract():
+    """Per-op operand requirements of moe_grouped_gemm_fp8 are checked on the
+    host, before any device work: the SiLU-backward GEMM needs its bf16 output
+    (its codes are made from it), and the wgrad GEMMs need 16-byte-aligned
+    scale arrays (they are bulk-copied)."""
+    from moe_expert_layer_replay_b200 import abi
+    L = abi.lib()
+    d = abi.dims(4096, 2048, 1024, 64, 6)
+    A = 0x100000  # aligned stand-ins; never dereferenced, every call fails its checks first
+    offs = ctypes.c_void_p(A)
+    g = abi.GemmArgs(A, A, A, A, A, A, A, None, None)  # b2 without out_bf16
+    assert L.moe_grouped_gemm_fp8(abi.GEMM_DGRAD_DOWN_SILU, ctypes.byref(d), offs, ctypes.byref(g), None) \
+        == abi.INVALID_ARG
+    for op in (abi.GEMM_WGRAD_DOWN, abi.GEMM_WGRAD_GATEUP):
+        g = abi.GemmArgs(A, A + 4, A, A, None, None, None, None, A)  # sa only 4-byte aligned
+        assert L.moe_grouped_gemm_fp8(op, ctypes.byref(d), offs, ctypes.byref(g), None) == abi.INVALID_ARG
+        g = abi.GemmArgs(A, A, A, A + 8, None, None, None, None, A)  # sb only 8-byte aligned
+        assert L.moe_grouped_gemm_fp8(op, ctypes.byref(d), offs, ctypes.byref(g), None) == abi.INVALID_ARG
+        g = abi.GemmArgs(A, A, A, A, None, None, None, None, None)  # no dW
+        assert L.moe_grouped_gemm_fp8(op, ctypes.byref(d), offs, ctypes.byref(g), None) == abi.INVALID_ARG
+    g = abi.GemmArgs(A, A, A, A, None, None, None, None, None)  # a7 without Y
+    assert L.moe_grouped_gemm_fp8(abi.GEMM_DOWN, ctypes.byref(d), offs, ctypes.byref(g), None) == abi.INVALID_ARG
+    assert L.moe_grouped_gemm_fp8(9, ctypes.byref(d), offs, ctypes.byref(g), None) == abi.INVALID_ARG
