@@ -52,7 +52,6 @@ int check_dims(const moe_dims *d, bool need_gemm_shapes)
     return MOE_OK;
 }
 
-int last_cuda() { return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
 }  // namespace
 
