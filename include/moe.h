@@ -103,7 +103,8 @@ int moe_route_topk(const float *logits, const moe_dims *dims, int32_t *idx, floa
 /* payload int32 [L][k][T] (element (l,j,t) at (l*k+j)*T+t) ->
  * idx[t][j] = payload[layer][j][t].  Weights: w_in [T][k] copied when non-NULL,
  * else softmax of the trainer logits [T][E] over the replayed set.  Exactly
- * one of w_in / logits must be non-NULL.  An entry outside [0,E) or an expert
+ * one of w_in / logits must be non-NULL (when T > 0; T = 0 does nothing and
+ * checks no array pointer).  An entry outside [0,E) or an expert
  * repeated within a token latches MOE_ERR_BAD_ROUTING; that token's weights
  * are 0 and its idx entries are copied as given (moe_permute drops entries
  * outside [0,E)). */
@@ -125,8 +126,10 @@ int moe_route_replay(const int32_t *payload, int32_t L, int32_t layer, const moe
  * With x (bf16 [T][D]) non-NULL, also dispatches x in FP8:
  *   xq [R_cap][D] e4m3, xs [D/128][R_cap] fp32: 1x128 blocks of row pos[t][j]
  *   are those of x[t]; padding rows get codes 0 and scale 0.
- *   xqT [D][R_cap], xsT [R_cap/128][D] (both nullable, align must be 128):
- *   128x1 blocks of the permuted rows, for the weight gradient.
+ *   xqT [D][R_cap], xsT [R_cap/128][D] (both nullable, align must be 128;
+ *   with T > 0 they need x): 128x1 blocks of the permuted rows, for the
+ *   weight gradient.  With T = 0 there is no row to dispatch and x may be
+ *   NULL (an empty array).
  * ws: moe_permute_workspace_size() bytes of scratch (16-byte aligned). */
 int moe_permute(const int32_t *idx, const moe_dims *dims, int32_t *counts, int32_t *offsets,
                 int32_t *pos, int32_t *src_idx, const uint16_t *x, uint8_t *xq, float *xs,

@@ -112,8 +112,9 @@ int moe_route_replay(const int32_t *payload, int32_t L, int32_t layer, const moe
     int st = check_dims(d, false);
     if (st) return st;
     if (L <= 0 || layer < 0 || layer >= L) return MOE_ERR_INVALID_ARG;
+    if (d->T == 0) return MOE_OK;  // nothing to replay (empty arrays may be null)
     if ((w_in == nullptr) == (logits == nullptr)) return MOE_ERR_INVALID_ARG;
-    if (d->T > 0 && (!payload || !idx || !w)) return MOE_ERR_INVALID_ARG;
+    if (!payload || !idx || !w) return MOE_ERR_INVALID_ARG;
     int *sp = status_ptr();
     if (!sp) return MOE_ERR_CUDA;
     return moe::launch_route_replay(payload, layer, d->T, d->E, d->k, w_in, logits, idx, w, sp,
@@ -131,7 +132,7 @@ int moe_permute(const int32_t *idx, const moe_dims *d, int32_t *counts, int32_t 
     if (ws_bytes < moe_permute_workspace_size(d) || !aligned16(ws)) return MOE_ERR_INVALID_ARG;
     if (x && (!xq || !xs || !aligned16(x) || !aligned16(xq) || !aligned4(xs))) return MOE_ERR_INVALID_ARG;
     if ((xqT == nullptr) != (xsT == nullptr)) return MOE_ERR_INVALID_ARG;
-    if (xqT && (!x || d->align != 128 || !aligned16(xqT))) return MOE_ERR_INVALID_ARG;
+    if (xqT && ((d->T > 0 && !x) || d->align != 128 || !aligned16(xqT))) return MOE_ERR_INVALID_ARG;
     int *sp = status_ptr();
     if (!sp) return MOE_ERR_CUDA;
     cudaStream_t s = as_stream(stream);

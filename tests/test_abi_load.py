@@ -64,3 +64,16 @@ def test_gemm_operand_contract():
     g = abi.GemmArgs(A, A, A, A, None, None, None, None, None)  # a7 without Y
     assert L.moe_grouped_gemm_fp8(abi.GEMM_DOWN, ctypes.byref(d), offs, ctypes.byref(g), None) == abi.INVALID_ARG
     assert L.moe_grouped_gemm_fp8(9, ctypes.byref(d), offs, ctypes.byref(g), None) == abi.INVALID_ARG
+
+
+def test_empty_batch_host_paths():
+    """T = 0: the entry points that have nothing to do return OK before any
+    device work, with the (empty, so NULL) arrays left unchecked."""
+    from moe_expert_layer_replay_b200 import abi
+    L = abi.lib()
+    d = abi.dims(0, 256, 128, 8, 2)
+    assert L.moe_route_replay(None, 4, 1, ctypes.byref(d), None, None, None, None, None) == abi.OK
+    assert L.moe_combine(None, None, None, ctypes.byref(d), None, None) == abi.OK
+    assert L.moe_unpermute_reduce(None, None, ctypes.byref(d), None, None) == abi.OK
+    # the layer index is still checked
+    assert L.moe_route_replay(None, 4, 4, ctypes.byref(d), None, None, None, None, None) == abi.INVALID_ARG

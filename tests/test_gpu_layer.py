@@ -212,3 +212,26 @@ def test_wait_budget_timeout_is_reported_and_recoverable(A):
     A.grouped_gemm_fp8(A.GEMM_GATEUP_SILU, d, B.offsets, B.xq, B.xs, W.wgu_q, W.wgu_s, out_q=B.hq, out_s=B.hs)
     assert A.get_status() == A.OK
     same_bits(host(B.hq)[:Rp], ref_hq[:Rp], "after a timed-out run")
+
+
+def test_empty_batch_forward_backward(A):
+    """T = 0 through the whole layer, top-k and replay routing alike: every
+    entry point returns OK, the outputs are empty, all segments are empty and
+    the weight gradients are untouched."""
+    from moe_expert_layer_replay_b200 import layer
+    T, D, I, E, k = 0, 256, 128, 8, 2
+    d = A.dims(T, D, I, E, k)
+    rng = np.random.default_rng(5)
+    W = layer.quantise_weights(d, dev(rand_bf16(rng, (E, I, D), 0.02)), dev(rand_bf16(rng, (E, I, D), 0.02)),
+                               dev(rand_bf16(rng, (E, D, I), 0.02)), train=True)
+    B = layer.Buffers(d, "cuda", train=True)
+    layer.route(B, logits=torch.empty(0, E, device="cuda"))
+    layer.route(B, payload=torch.empty(1, k, 0, dtype=torch.int32, device="cuda"), layer=0,
+                w_in=torch.empty(0, k, device="cuda"))
+    y = layer.forward(B, torch.empty(0, D, dtype=torch.bfloat16, device="cuda"), W)
+    dx, d_w, dz = layer.backward(B, torch.empty(0, D, dtype=torch.bfloat16, device="cuda"), W, router_logits=True)
+    torch.cuda.synchronize()
+    assert A.get_status() == A.OK
+    assert y.shape == (0, D) and dx.shape == (0, D) and d_w.shape == (0, k) and dz.shape == (0, E)
+    assert int(B.counts.abs().sum()) == 0 and int(B.offsets.abs().sum()) == 0
+    assert int(torch.count_nonzero(B.dWd)) == 0 and int(torch.count_nonzero(B.dWgu)) == 0
