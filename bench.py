@@ -272,8 +272,9 @@ def run_ours(args, wl_name):
 
     launches_per_step = wl.L * (1 + 4 + 1 + 1 + 1)  # replay, permute (count/scan/place/dispatch quant), 2 GEMMs, combine
 
-    clocks = Clocks(local, os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv")) \
-        if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else Clocks(local, f"/tmp/moe_clocks_{rank}.csv")
+    import tempfile
+    clocks_dir = os.environ.get("MOE_BENCH_CLOCKS_DIR", tempfile.gettempdir())  # raw nvidia-smi samples
+    clocks = Clocks(local, os.path.join(clocks_dir, f"moe_clocks_rank{rank}.csv"))
     clocks.mark()
     for _ in range(max(3, args.warmup)):
         step(False)

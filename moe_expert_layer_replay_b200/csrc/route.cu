@@ -59,7 +59,7 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict
             my_e = be;
         }
     }
-    // softmax over the chosen set; round 0 holds the largest logit
+    // softmax over the chosen set; the first selection holds the largest logit
     float m = __shfl_sync(kFull, my_v, 0);
     float ex = (lane < k) ? expf(my_v - m) : 0.0f;
     float sum = ex;
@@ -115,7 +115,7 @@ __global__ void __launch_bounds__(128) route_topk_small_kernel(const float *__re
             se[j] = be;
         }
     }
-    // softmax over the chosen set; round 0 holds the largest logit
+    // softmax over the chosen set; the first selection holds the largest logit
     float ex[16], sum = 0.0f;
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
