@@ -86,6 +86,11 @@ int moe_get_status(void *stream, int *out);
  * memory and returns. */
 void moe_set_wait_budget(uint64_t cycles);
 
+/* Number of kernels this library has launched in this process, counting a
+ * launch recorded into a stream capture once (a graph replay launches them
+ * again without calling into the library).  For accounting only. */
+uint64_t moe_kernel_launches(void);
+
 /* ------------------------------------------------------------------------ */
 /* a1  Top-k routing  [P1 §Drift og omkostninger i realiteten]               */
 /* ------------------------------------------------------------------------ */
@@ -146,7 +151,9 @@ int moe_permute(const int32_t *idx, const moe_dims *dims, int32_t *counts, int32
  * MOE_ERR_UNSUPPORTED.  The first call on a device looks up the array's
  * address (make it before any stream capture); calls overlapping on the GPU
  * share the array and race; entries outside [0,E) are dropped (pos = -1) but
- * not reported through moe_get_status(). */
+ * not reported through moe_get_status().  The address is kept for the life of
+ * the process: after cudaDeviceReset() on a device, do not call this entry
+ * point on that device again in the same process. */
 int moe_permute_noalloc(const int32_t *idx, const moe_dims *dims, int32_t *counts, int32_t *offsets,
                         int32_t *pos, int32_t *src_idx, const uint16_t *x, uint8_t *xq, float *xs,
                         void *stream);

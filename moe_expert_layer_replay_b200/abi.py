@@ -20,7 +20,7 @@ EXPORTS = [
     "moe_rows_capacity", "moe_permute_workspace_size", "moe_strerror", "moe_get_status",
     "moe_set_wait_budget", "moe_route_topk", "moe_route_replay", "moe_permute",
     "moe_quant_fp8_block", "moe_quant_weights", "moe_grouped_gemm_fp8", "moe_combine",
-    "moe_combine_bwd", "moe_unpermute_reduce", "moe_permute_noalloc",
+    "moe_combine_bwd", "moe_unpermute_reduce", "moe_permute_noalloc", "moe_kernel_launches",
 ]
 
 
@@ -63,6 +63,7 @@ def lib() -> ctypes.CDLL:
             "moe_strerror": (ctypes.c_char_p, [ctypes.c_int]),
             "moe_get_status": (ctypes.c_int, [P, ctypes.POINTER(ctypes.c_int)]),
             "moe_set_wait_budget": (None, [U64]),
+            "moe_kernel_launches": (U64, []),
             "moe_route_topk": (ctypes.c_int, [P, D, P, P, P]),
             "moe_route_replay": (ctypes.c_int, [P, I32, I32, D, P, P, P, P, P]),
             "moe_permute": (ctypes.c_int, [P, D, P, P, P, P, P, P, P, P, P, P, SZ, P]),
@@ -126,6 +127,11 @@ def get_status(stream=None) -> int:
 
 def set_wait_budget(cycles: int) -> None:
     lib().moe_set_wait_budget(int(cycles))
+
+
+def kernel_launches() -> int:
+    """Kernels launched (or recorded into a capture) by the library so far."""
+    return int(lib().moe_kernel_launches())
 
 
 # ------------------------------------------------------------ entry points --

@@ -67,6 +67,7 @@ int launch_combine(const uint16_t *Y, const float *w, const int32_t *pos, int T,
         gather_reduce_kernel<true><<<blocks, 256, 0, s>>>(Y, w, pos, T, D, k, y);
     else
         gather_reduce_kernel<false><<<blocks, 256, 0, s>>>(Y, nullptr, pos, T, D, k, y);
+    count_launch();
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -184,6 +185,7 @@ int launch_combine_bwd(const uint16_t *dy, const uint16_t *Y, const float *w, co
     if (T == 0) return MOE_OK;
     combine_bwd_kernel<<<(unsigned)((T + 7) / 8), 256, 0, s>>>(dy, Y, w, pos, idx, T, D, k, E, R_cap,
                                                                dYq, dYs, dYb, d_w, d_logits);
+    count_launch();
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

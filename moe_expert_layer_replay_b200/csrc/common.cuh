@@ -175,6 +175,9 @@ __device__ __forceinline__ float absmax8(const float *v, float m)
 
 // Launchers (host side, one per kernel family), defined in the .cu files.
 namespace moe {
+// Counts one kernel launch (or one launch recorded into a stream capture);
+// read by moe_kernel_launches().
+void count_launch();
 int launch_route_topk(const float *z, int T, int E, int k, int32_t *idx, float *w, cudaStream_t s);
 int launch_route_replay(const int32_t *P, int layer, int T, int E, int k, const float *w_in,
                         const float *z, int32_t *idx, float *w, int *status, cudaStream_t s);

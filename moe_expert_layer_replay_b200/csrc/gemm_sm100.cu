@@ -837,6 +837,7 @@ static int launch_one(const CUtensorMap &a, const CUtensorMap &b, const CUtensor
         configured = true;
     }
     gemm::grouped_gemm_kernel<kEpi><<<grid, gemm::NUM_THREADS, gemm::smem_bytes<kEpi>(), s>>>(a, b, c, args);
+    count_launch();
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

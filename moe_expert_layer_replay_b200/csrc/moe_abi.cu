@@ -3,6 +3,8 @@
 // include/moe.h.
 #include <stdio.h>
 
+#include <atomic>
+
 #include "common.cuh"
 
 namespace moe {
@@ -12,6 +14,12 @@ int launch_grouped_gemm(int op, const moe_dims &d, int64_t R_cap, const int32_t 
 
 // Latched device status word (one per device that loads the library).
 static __device__ int g_moe_status;
+
+namespace {
+std::atomic<uint64_t> g_launches{0};
+}
+
+void moe::count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 namespace {
 
@@ -97,6 +105,8 @@ int moe_get_status(void *stream, int *out)
 }
 
 void moe_set_wait_budget(uint64_t cycles) { g_wait_budget = cycles; }
+
+uint64_t moe_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
 
 int moe_route_topk(const float *logits, const moe_dims *d, int32_t *idx, float *w, void *stream)
 {

@@ -202,6 +202,7 @@ int launch_permute_index(const int32_t *idx, int T, int k, int E, int align, int
     int32_t *blkbase = blkcnt + (int64_t)(nblk ? nblk : 1) * E;
     if (nblk > 0) {
         perm_count_kernel<<<nblk, 256, E * sizeof(int), s>>>(idx, n, E, blkcnt);
+        count_launch();
     }
     // place also writes -1 to the rows of src_idx that no entry fills; with
     // few blocks it does the scan pass itself (one launch less)
@@ -210,10 +211,13 @@ int launch_permute_index(const int32_t *idx, int T, int k, int E, int align, int
     if (nblk <= 64) {
         perm_place_kernel<true><<<pblk, 32 * kPlaceWarps, psmem, s>>>(idx, n, E, align, nblk, blkcnt, blkbase,
                                                                      offsets, counts, R_cap, pos, src_idx, status);
+        count_launch();
     } else {
         perm_scan_kernel<<<1, 256, 0, s>>>(blkcnt, nblk, E, align, blkbase, counts, offsets);
+        count_launch();
         perm_place_kernel<false><<<pblk, 32 * kPlaceWarps, psmem, s>>>(idx, n, E, align, nblk, blkcnt, blkbase,
                                                                       offsets, counts, R_cap, pos, src_idx, status);
+        count_launch();
     }
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -22,6 +22,12 @@
 //    so nothing needs clearing.
 //  - A problem needing more scratch than the array holds is rejected with
 //    MOE_ERR_UNSUPPORTED before anything is launched.
+//  - The looked-up address is kept for the life of the process.  After a
+//    cudaDeviceReset() the module is loaded again and the array may move, so
+//    a process that resets a device must not call this entry point on it
+//    again (use moe_permute with its own workspace, or a fresh process).
+#include <atomic>
+
 #include "common.cuh"
 
 namespace {
@@ -32,21 +38,23 @@ constexpr size_t kScratchBytes = 1u << 20;
 static __device__ __align__(256) unsigned char g_permute_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
-void *g_scratch_addr[kMaxDevices];
+std::atomic<void *> g_scratch_addr[kMaxDevices];
 
 // Device address of the scratch array for the current device, looked up once
 // per device with that device current.  (In host code the array's name is
-// only a host-side stand-in, never a device address.)
+// only a host-side stand-in, never a device address.)  Host threads that make
+// their first call on a device at the same time may both look it up; they
+// find the same address, and the slot is atomic.
 int scratch_address(void **scratch)
 {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
-    if (!g_scratch_addr[dev]) {
-        void *p = nullptr;
+    void *p = g_scratch_addr[dev].load(std::memory_order_acquire);
+    if (!p) {
         if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess || !p) return MOE_ERR_CUDA;
-        g_scratch_addr[dev] = p;
+        g_scratch_addr[dev].store(p, std::memory_order_release);
     }
-    *scratch = g_scratch_addr[dev];
+    *scratch = p;
     return MOE_OK;
 }
 

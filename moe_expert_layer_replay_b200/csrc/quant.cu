@@ -103,6 +103,7 @@ int launch_quant_1x128(const uint16_t *in, int64_t ld, int64_t rows, int64_t col
     int64_t blocks = (rows + 7) / 8;
     quant_1x128_kernel<false><<<(unsigned)blocks, 256, 0, s>>>(in, ld, rows, cols, pos, k, q, ldq, sc, ld_s,
                                                                nullptr, nullptr, 0);
+    count_launch();
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -114,6 +115,7 @@ int launch_dispatch_quant(const uint16_t *x, int64_t T, int64_t D, const int32_t
     const int64_t warps = T + (int64_t)E * kPadWarps;
     quant_1x128_kernel<true><<<(unsigned)((warps + 7) / 8), 256, 0, s>>>(x, D, T, D, pos, k, xq, D, xs, R_cap,
                                                                         counts, offsets, E);
+    count_launch();
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -188,6 +190,7 @@ int launch_quant_rows128(const uint16_t *in, int64_t ld, const int32_t *src_idx,
     if (rows == 0 || cols == 0) return MOE_OK;
     dim3 grid((unsigned)((rows + 127) / 128), (unsigned)((cols + 63) / 64));
     quant_rows128_kernel<<<grid, 256, 0, s>>>(in, ld, src_idx, k, rows, cols, ld_rows, qT, sT);
+    count_launch();
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -224,6 +227,7 @@ int launch_pad_rows(const int32_t *counts, const int32_t *offsets, int E, int64_
 {
     if (E == 0) return MOE_OK;
     pad_rows_kernel<<<E, 256, 0, s>>>(counts, offsets, cols, R_cap, q, sc, bf);
+    count_launch();
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -318,6 +322,7 @@ int launch_quant_128x128(const uint16_t *in, int64_t rows, int64_t cols, int64_t
     quant_128x128_kernel<<<grid, 256, 0, s>>>(in, rows, cols, ld, in_expert_stride, rb_mul, rb_add, q,
                                               q_expert_stride, sc, s_expert_stride, qT, qT_ld,
                                               qT_expert_stride, sT, sT_ld, sT_expert_stride);
+    count_launch();
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

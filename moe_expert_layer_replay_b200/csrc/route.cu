@@ -203,9 +203,11 @@ int launch_route_topk(const float *z, int T, int E, int k, int32_t *idx, float *
     if (T == 0) return MOE_OK;
     if (E <= 32) {
         route_topk_small_kernel<<<(T + 127) / 128, 128, 0, s>>>(z, T, E, k, idx, w);
+        count_launch();
     } else {
         const int blocks = (T + 7) / 8;
         route_topk_kernel<<<blocks, 256, 0, s>>>(z, T, E, k, idx, w);
+        count_launch();
     }
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
@@ -215,6 +217,7 @@ int launch_route_replay(const int32_t *P, int layer, int T, int E, int k, const 
 {
     if (T == 0) return MOE_OK;
     route_replay_kernel<<<(T + 63) / 64, 64, 0, s>>>(P, layer, T, E, k, w_in, z, idx, w, status);
+    count_launch();
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

@@ -11,7 +11,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 def test_reference_arm_json_line():
     out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
-                          "--warmup", "0", "--ref-tokens", "8"], capture_output=True, text=True, timeout=600,
+                          "--warmup", "0", "--ref-tokens", "8", "--workload", "replay"], capture_output=True,
+                         text=True, timeout=600,
                          cwd=ROOT, env={**os.environ, "RANK": "0"})
     assert out.returncode == 0, out.stderr[-2000:]
     lines = [l for l in out.stdout.splitlines() if l.startswith("{")]
@@ -31,3 +32,17 @@ def test_reference_arm_other_ranks_exit_quietly():
                           "--warmup", "0", "--ref-tokens", "8"], capture_output=True, text=True, timeout=120,
                          cwd=ROOT, env={**os.environ, "RANK": "1"})
     assert out.returncode == 0 and not [l for l in out.stdout.splitlines() if l.startswith("{")]
+
+
+def test_default_workload_is_the_largest_single_gpu_configuration():
+    """With no flags the bench times the long-sequence prefill chunk (T=131072,
+    d_model=6144, I=2048, 32 experts, top-8, skewed routing with empty
+    experts), the largest configuration of the layer on one GPU."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from moe_expert_layer_replay_b200.inputs import WORKLOADS
+    args = bench.build_parser().parse_args([])
+    wl = WORKLOADS[args.workload]
+    assert (wl.T, wl.D, wl.I, wl.E, wl.k, wl.empty) == (131072, 6144, 2048, 32, 8, 4)
+    assert args.gpus == 1 and args.warmup >= 3 and args.impl == "ours"
+    assert bench.default_sample_tokens(wl, 3e11) <= 512

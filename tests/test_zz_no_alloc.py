@@ -23,15 +23,25 @@ def _case(rng, T, E, k, zipf):
     return np.argsort(-keys, axis=1, kind="stable")[:, :k].astype(np.int32)
 
 
-def test_permute_noalloc_matches_permute_twice():
+# (T, E, k, D, zipf, align), in call order: each smaller problem follows a
+# larger one, so a call finds the array holding a bigger call's contents.  The
+# first and third have more than 64 chunks of routed entries, which runs the
+# separate count, scan and place passes (block bases written by one kernel
+# into the array and read by the next); the others run the fused place pass.
+CASES = [(16384, 32, 8, 256, 1.2, 128), (4096, 64, 6, 512, 1.1, 128), (20000, 16, 4, 128, 0.0, 1),
+         (3000, 32, 8, 256, 0.5, 1)]
+
+
+def test_permute_noalloc_matches_permute_and_oracle(orc):
+    from oracle import layer as OL
     from moe_expert_layer_replay_b200 import abi, build
     build.build()
     A = abi
-    for call, (T, E, k, D, zipf) in enumerate([(4096, 64, 6, 512, 1.1), (3000, 32, 8, 256, 0.5)]):
+    for call, (T, E, k, D, zipf, align) in enumerate(CASES):
         rng = np.random.default_rng(40 + call)
         idx = _case(rng, T, E, k, zipf)
         x = rand_bf16(rng, (T, D))
-        d = A.dims(T, D, 128, E, k, 128)
+        d = A.dims(T, D, 128, E, k, align)
         R = A.rows_capacity(d)
         outs = []
         for noalloc in (False, True):
@@ -48,7 +58,15 @@ def test_permute_noalloc_matches_permute_twice():
             Rp = int(host(offsets)[E])
             outs.append([host(counts), host(offsets), host(pos), host(src), host(xq)[:Rp], host(xs)[:, :Rp]])
         for a, b, name in zip(outs[0], outs[1], ["counts", "offsets", "pos", "src_idx", "xq", "xs"]):
-            same_bits(b, a, f"call {call}: {name}")
+            same_bits(b, a, f"call {call}: {name} (no-alloc vs workspace)")
+        # and both against the oracle
+        oc, oo, op, osrc = orc.permute(idx, E, align, R)
+        for got, ref, name in zip(outs[1][:4], [oc, oo, op, osrc], ["counts", "offsets", "pos", "src_idx"]):
+            same_bits(got, ref, f"call {call}: {name} (oracle)")
+        Rp = int(oo[E])
+        q_ref, s_ref = orc.quant_block(OL.dispatch_rows(x, osrc, np.arange(Rp), k), 1, 128)
+        same_bits(outs[1][4], q_ref, f"call {call}: xq (oracle)")
+        same_bits(outs[1][5].T, s_ref, f"call {call}: xs (oracle)")
 
 
 def test_permute_noalloc_rejects_oversize():
