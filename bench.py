@@ -58,7 +58,7 @@ GEMM1_TRAFFIC = {
 def _gemm_sources_hash() -> str:
     import hashlib
     h = hashlib.sha256()
-    for f in ("gemm_sm100.cu", "common.cuh"):
+    for f in ("gemm_sm100.cu", "sm100.cuh", "common.cuh"):
         with open(os.path.join(ROOT, "moe_expert_layer_replay_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]

@@ -103,6 +103,41 @@ int moe_route_topk(const float *logits, const moe_dims *dims, int32_t *idx, floa
                    void *stream);
 
 /* ------------------------------------------------------------------------ */
+/* Router and capture of its decisions  [P1 §Drift og omkostninger;          */
+/* P4 §Router Replay]                                                        */
+/* ------------------------------------------------------------------------ */
+/* The router is the linear gate before the top-k: x bf16 [T][D], w_r bf16
+ * [E][D] -> z fp32 [T][E], z[t][e] = sum_d x[t][d] w_r[e][d] (bf16 products
+ * accumulated in fp32 on the tensor cores; the order of the additions is the
+ * hardware's).  With idx and w non-NULL (both or neither) it then chooses
+ * idx/w from z exactly as moe_route_topk does.  D % 128 == 0, E <= 256;
+ * x, w_r and z 16-byte aligned. */
+int moe_router_fwd(const uint16_t *x, const uint16_t *w_r, const moe_dims *dims, float *z, int32_t *idx,
+                   float *w, void *stream);
+
+/* Capture: writes the routing decisions of one layer into the replay
+ * payload, payload[layer][j][t] = idx[t][j] (int32 [L][k][T], element
+ * (l,j,t) at (l*k+j)*T+t: the layout moe_route_replay reads).  Other layers'
+ * slices are untouched. */
+int moe_capture_payload(const int32_t *idx, const moe_dims *dims, int32_t L, int32_t layer, int32_t *payload,
+                        void *stream);
+
+/* Bytes of caller-provided scratch for moe_router_bwd's weight gradient. */
+size_t moe_router_bwd_workspace_size(const moe_dims *dims);
+
+/* Router backward from the logit gradient dz fp32 [T][E] (moe_combine_bwd's
+ * d_logits):
+ *   dx bf16 [T][D] (nullable: skipped) = bf16(fp32(dx_in[t][d]) +
+ *        sum_e dz[t][e] w_r[e][d]), sum in fp32, e ascending; dx_in nullable
+ *        (0) and may equal dx (the router's share added in place);
+ *   dw_r fp32 [E][D] (nullable: skipped) += sum_t dz[t][e] x[t][d]: fp32
+ *        partial sums over 256-token chunks (tokens in order) in ws, then
+ *        added chunk by chunk in order (deterministic).
+ * ws: moe_router_bwd_workspace_size() bytes, 16-byte aligned (only for dw_r). */
+int moe_router_bwd(const float *dz, const uint16_t *x, const uint16_t *w_r, const moe_dims *dims,
+                   const uint16_t *dx_in, uint16_t *dx, float *dw_r, void *ws, size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------ */
 /* a2  Router replay  [P4 §Router Replay]                                    */
 /* ------------------------------------------------------------------------ */
 /* payload int32 [L][k][T] (element (l,j,t) at (l*k+j)*T+t) ->

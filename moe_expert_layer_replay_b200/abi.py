@@ -21,6 +21,7 @@ EXPORTS = [
     "moe_set_wait_budget", "moe_route_topk", "moe_route_replay", "moe_permute",
     "moe_quant_fp8_block", "moe_quant_weights", "moe_grouped_gemm_fp8", "moe_combine",
     "moe_combine_bwd", "moe_unpermute_reduce", "moe_permute_noalloc", "moe_kernel_launches",
+    "moe_router_fwd", "moe_capture_payload", "moe_router_bwd_workspace_size", "moe_router_bwd",
 ]
 
 
@@ -66,6 +67,10 @@ def lib() -> ctypes.CDLL:
             "moe_kernel_launches": (U64, []),
             "moe_route_topk": (ctypes.c_int, [P, D, P, P, P]),
             "moe_route_replay": (ctypes.c_int, [P, I32, I32, D, P, P, P, P, P]),
+            "moe_router_fwd": (ctypes.c_int, [P, P, D, P, P, P, P]),
+            "moe_capture_payload": (ctypes.c_int, [P, D, I32, I32, P, P]),
+            "moe_router_bwd_workspace_size": (SZ, [D]),
+            "moe_router_bwd": (ctypes.c_int, [P, P, P, D, P, P, P, P, SZ, P]),
             "moe_permute": (ctypes.c_int, [P, D, P, P, P, P, P, P, P, P, P, P, SZ, P]),
             "moe_permute_noalloc": (ctypes.c_int, [P, D, P, P, P, P, P, P, P, P]),
             "moe_quant_fp8_block": (ctypes.c_int, [P, I64, I64, I64, I32, I32, P, P, P, P, P]),
@@ -142,6 +147,25 @@ def route_topk(logits, d: Dims, idx, w, stream=None):
 def route_replay(payload, L, layer, d: Dims, w_in, logits, idx, w, stream=None):
     _check("moe_route_replay", lib().moe_route_replay(_p(payload), int(L), int(layer), ctypes.byref(d),
                                                       _p(w_in), _p(logits), _p(idx), _p(w), _s(stream)))
+
+
+def router_fwd(x, w_r, d: Dims, z, idx=None, w=None, stream=None):
+    _check("moe_router_fwd", lib().moe_router_fwd(_p(x), _p(w_r), ctypes.byref(d), _p(z), _p(idx), _p(w), _s(stream)))
+
+
+def capture_payload(idx, d: Dims, L, layer, payload, stream=None):
+    _check("moe_capture_payload", lib().moe_capture_payload(_p(idx), ctypes.byref(d), int(L), int(layer),
+                                                            _p(payload), _s(stream)))
+
+
+def router_bwd_workspace_size(d: Dims) -> int:
+    return int(lib().moe_router_bwd_workspace_size(ctypes.byref(d)))
+
+
+def router_bwd(dz, x, w_r, d: Dims, dx_in=None, dx=None, dw_r=None, ws=None, stream=None):
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check("moe_router_bwd", lib().moe_router_bwd(_p(dz), _p(x), _p(w_r), ctypes.byref(d), _p(dx_in), _p(dx),
+                                                  _p(dw_r), _p(ws), nbytes, _s(stream)))
 
 
 def permute(idx, d: Dims, counts, offsets, pos, src_idx, x, xq, xs, xqT, xsT, ws, stream=None):

@@ -201,6 +201,12 @@ int launch_quant_128x128(const uint16_t *in, int64_t rows, int64_t cols, int64_t
                          int64_t q_expert_stride, float *sc, int64_t s_expert_stride, uint8_t *qT,
                          int64_t qT_ld, int64_t qT_expert_stride, float *sT, int64_t sT_ld,
                          int64_t sT_expert_stride, cudaStream_t s);
+size_t router_bwd_ws_bytes(int T, int D, int E);
+int launch_router_logits(const uint16_t *x, const uint16_t *w_r, int T, int D, int E, float *z, int *status,
+                         uint64_t budget, cudaStream_t s);
+int launch_capture(const int32_t *idx, int T, int k, int layer, int32_t *payload, cudaStream_t s);
+int launch_router_bwd(const float *dz, const uint16_t *x, const uint16_t *w_r, int T, int D, int E,
+                      const uint16_t *dx_in, uint16_t *dx, float *dw_r, void *ws, cudaStream_t s);
 int launch_combine(const uint16_t *Y, const float *w, const int32_t *pos, int T, int D, int k,
                    uint16_t *y, cudaStream_t s);
 int launch_combine_bwd(const uint16_t *dy, const uint16_t *Y, const float *w, const int32_t *pos,

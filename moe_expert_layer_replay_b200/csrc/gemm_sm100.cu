@@ -31,10 +31,7 @@
 //
 // Every mbarrier wait is bounded; on expiry the kernel latches
 // MOE_ERR_TIMEOUT, drains the copies and MMAs it issued, frees TMEM and exits.
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
-#include "common.cuh"
+#include "sm100.cuh"
 
 namespace moe {
 
@@ -47,7 +44,6 @@ constexpr int NUM_THREADS = 384;
 constexpr int EPI_WARP0 = 4;
 constexpr int EPI_THREADS = 256;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint64_t DRAIN_BUDGET = 1ull << 28;
 // smem: operand ring | barriers (full[4], empty[4], tfull[2], tempty[2], drain, epi) |
 // tmem slot | abort flag | offsets[257] | then, 1024-aligned, a region whose
 // use depends on the epilogue:
@@ -105,140 +101,7 @@ struct Args {
 };
 
 // ----------------------------------------------------------------- PTX ----
-__device__ __forceinline__ uint32_t smem_u32(const void *p)
-{
-    return (uint32_t)__cvta_generic_to_shared(p);
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
-{
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.b32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes)
-{
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-                 : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint32_t bar)
-{
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-
-// Bounded wait.  Returns false when the CTA is aborting (flag set by any role)
-// or when this wait ran out (then it sets the flag and latches the status).
-__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, uint64_t budget,
-                                             volatile int *abort_flag, int *status)
-{
-    if (mbar_try_wait(bar, parity)) return true;
-    const long long t0 = clock64();
-    for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((uint64_t)(clock64() - t0) > budget) {
-            *abort_flag = 1;
-            latch_status(status, MOE_ERR_TIMEOUT);
-            return false;
-        }
-        if ((it & 7u) == 0 && *abort_flag) return false;  // another role gave up
-    }
-}
-
-// Warp-wide wait: lane 0 polls, the other lanes wait for its verdict.
-__device__ __forceinline__ bool warp_wait_bounded(uint32_t bar, uint32_t parity, uint64_t budget,
-                                                  volatile int *abort_flag, int *status)
-{
-    bool ok = true;
-    if ((threadIdx.x & 31) == 0) ok = wait_bounded(bar, parity, budget, abort_flag, status);
-    return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-}
-
-// Drain wait: ignores the abort flag (used on the way out).
-__device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity)
-{
-    const long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity))
-        if ((uint64_t)(clock64() - t0) > DRAIN_BUDGET) return;
-}
-
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int32_t c0,
-                                            int32_t c1, uint32_t bar)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
-        : "memory");
-}
-
-// Bulk copy global -> shared (16-byte aligned, size a multiple of 16),
-// completing on an mbarrier's transaction count.
-__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar)
-{
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-                 "l"(src), "r"(bytes), "r"(bar)
-                 : "memory");
-}
-
-__device__ __forceinline__ void cp_async4(void *dst, const void *src)
-{
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int n>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(n) : "memory"); }
-
-// a = fma(p, s, a) on two fp32 lanes at once (packed f32x2)
-__device__ __forceinline__ void ffma2(float &a0, float &a1, float p0, float p1, float s0, float s1)
-{
-    asm("{\n\t.reg .b64 a, p, q;\n\tmov.b64 a, {%0, %1};\n\tmov.b64 p, {%2, %3};\n\t"
-        "mov.b64 q, {%4, %5};\n\tfma.rn.f32x2 a, p, q, a;\n\tmov.b64 {%0, %1}, a;\n\t}"
-        : "+f"(a0), "+f"(a1)
-        : "f"(p0), "f"(p1), "f"(s0), "f"(s1));
-}
-
-// TMA store of a 2D box from shared memory (bulk-group completion).
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t src, int32_t c0, int32_t c1)
-{
-    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
-                     reinterpret_cast<uint64_t>(map)),
-                 "r"(src), "r"(c0), "r"(c1)
-                 : "memory");
-}
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-template <int n>
-__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(n) : "memory"); }
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
-// 1024 bytes apart (SBO), version 1 (sm_100), base offset 0 (1024-aligned).
-__device__ __forceinline__ uint64_t sdesc(uint32_t saddr)
-{
-    uint64_t d = 0;
-    d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
-    d |= (uint64_t)1 << 16;             // leading byte offset (unused when swizzled)
-    d |= (uint64_t)(1024 >> 4) << 32;   // stride byte offset
-    d |= (uint64_t)1 << 46;             // descriptor version
-    d |= (uint64_t)2 << 61;             // SWIZZLE_128B
-    return d;
-}
+using namespace sm100;
 
 // Instruction descriptor, kind::f8f6f4: D fp32, A and B e4m3, both K-major,
 // N = 256, M = 128.
@@ -253,26 +116,6 @@ __device__ __forceinline__ void mma_f8(uint32_t tmem_d, uint64_t a, uint64_t b, 
         "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
         "l"(a), "l"(b), "r"(IDESC), "r"(accum));
 }
-
-__device__ __forceinline__ void mma_commit(uint32_t bar)
-{
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-                 : "memory");
-}
-
-#define MOE_TMEM_LD32(taddr, r)                                                                        \
-    asm volatile(                                                                                      \
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"   \
-        "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"                 \
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),          \
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),      \
-          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),   \
-          "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),   \
-          "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])                                           \
-        : "r"(taddr))
-
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-
 
 // ------------------------------------------------------------ schedule ----
 struct Tile {
@@ -771,59 +614,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 }  // namespace gemm
 
 // ------------------------------------------------------------------ host ----
-static PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn()
-{
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        cudaDriverEntryPointQueryResult q;
-        void *ptr = nullptr;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    }
-    return fn;
-}
-
-// 2D uint8 tensor [rows][cols] (row stride cols bytes), box box_rows x 128
-// bytes, 128-byte swizzle; out-of-range elements read as zero.
-static bool make_map(CUtensorMap *map, const void *base, uint64_t cols, uint64_t rows, uint32_t box_rows)
-{
-    auto fn = get_encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {cols};
-    cuuint32_t box[2] = {128, box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
-// Row-major [rows][cols] output of 1- or 2-byte elements, boxes of 32 rows x
-// 64 bytes, no swizzle (TMA stores of the SiLU and bf16 epilogues).
-static bool make_store_map(CUtensorMap *map, void *base, uint64_t cols, uint64_t rows, int esize)
-{
-    auto fn = get_encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {cols * esize};
-    cuuint32_t box[2] = {(cuuint32_t)(64 / esize), 32};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(map, esize == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base,
-                    dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
-static int sm_count()
-{
-    int dev = 0, n = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    return n > 0 ? n : 148;
-}
+using namespace sm100;
 
 template <int kEpi>
 static int launch_one(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &c, const gemm::Args &args,

@@ -31,6 +31,7 @@ cudaStream_t as_stream(void *s) { return reinterpret_cast<cudaStream_t>(s); }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+bool aligned8(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 7u) == 0; }
 
 // Device address of the status word for the current device (looked up once
 // per device, with that device current).
@@ -129,6 +130,53 @@ int moe_route_replay(const int32_t *payload, int32_t L, int32_t layer, const moe
     if (!sp) return MOE_ERR_CUDA;
     return moe::launch_route_replay(payload, layer, d->T, d->E, d->k, w_in, logits, idx, w, sp,
                                     as_stream(stream));
+}
+
+int moe_router_fwd(const uint16_t *x, const uint16_t *w_r, const moe_dims *d, float *z, int32_t *idx, float *w,
+                   void *stream)
+{
+    int st = check_dims(d, false);
+    if (st) return st;
+    if (d->T == 0) return MOE_OK;
+    if (!x || !w_r || !z || !aligned16(x) || !aligned16(w_r) || !aligned16(z)) return MOE_ERR_INVALID_ARG;
+    if ((idx == nullptr) != (w == nullptr)) return MOE_ERR_INVALID_ARG;
+    int *sp = status_ptr();
+    if (!sp) return MOE_ERR_CUDA;
+    cudaStream_t s = as_stream(stream);
+    st = moe::launch_router_logits(x, w_r, d->T, d->D, d->E, z, sp, wait_budget(), s);
+    if (st || !idx) return st;
+    return moe::launch_route_topk(z, d->T, d->E, d->k, idx, w, s);
+}
+
+int moe_capture_payload(const int32_t *idx, const moe_dims *d, int32_t L, int32_t layer, int32_t *payload,
+                        void *stream)
+{
+    int st = check_dims(d, false);
+    if (st) return st;
+    if (L <= 0 || layer < 0 || layer >= L) return MOE_ERR_INVALID_ARG;
+    if (d->T == 0) return MOE_OK;
+    if (!idx || !payload) return MOE_ERR_INVALID_ARG;
+    return moe::launch_capture(idx, d->T, d->k, layer, payload, as_stream(stream));
+}
+
+size_t moe_router_bwd_workspace_size(const moe_dims *d)
+{
+    if (!d || d->T < 0 || d->D <= 0 || d->E <= 0) return 0;
+    return moe::router_bwd_ws_bytes(d->T, d->D, d->E);
+}
+
+int moe_router_bwd(const float *dz, const uint16_t *x, const uint16_t *w_r, const moe_dims *d,
+                   const uint16_t *dx_in, uint16_t *dx, float *dw_r, void *ws, size_t ws_bytes, void *stream)
+{
+    int st = check_dims(d, false);
+    if (st) return st;
+    if (d->T == 0) return MOE_OK;
+    if (!dz) return MOE_ERR_INVALID_ARG;
+    if (dx && (!w_r || !aligned4(w_r) || !aligned4(dx) || (dx_in && !aligned4(dx_in)))) return MOE_ERR_INVALID_ARG;
+    if (dw_r && (!x || !aligned4(x) || !aligned8(dw_r) || !ws || ws_bytes < moe_router_bwd_workspace_size(d) ||
+                 !aligned16(ws)))
+        return MOE_ERR_INVALID_ARG;
+    return moe::launch_router_bwd(dz, x, w_r, d->T, d->D, d->E, dx_in, dx, dw_r, ws, as_stream(stream));
 }
 
 int moe_permute(const int32_t *idx, const moe_dims *d, int32_t *counts, int32_t *offsets,
