@@ -272,6 +272,18 @@ typedef struct {
 int moe_grouped_gemm_fp8(int32_t op, const moe_dims *dims, const int32_t *offsets,
                          const moe_gemm_args *args, void *stream);
 
+/* The same GEMMs (rows-mode ops only: GATEUP_SILU, DOWN, DGRAD_DOWN_SILU,
+ * DGRAD_GATEUP) over n_seg 128-aligned row segments offsets[0..n_seg] that
+ * are not one per expert: segment v uses the weights of expert v % dims->E
+ * (dims->E experts in the weight arrays; n_seg a multiple of it, <= 256).
+ * rows_cap (a multiple of 128) replaces moe_rows_capacity(dims) as the row
+ * count of every row-indexed operand and the leading dimension of the 1x128
+ * scale arrays; dims->T and dims->k are not used.  This is the layout an
+ * expert-parallel rank receives: one segment per (source rank, local expert)
+ * [P4 §Parallelism/EP, §Wide Expert Parallelism]. */
+int moe_grouped_gemm_fp8_seg(int32_t op, const moe_dims *dims, int64_t rows_cap, const int32_t *offsets,
+                             int32_t n_seg, const moe_gemm_args *args, void *stream);
+
 /* ------------------------------------------------------------------------ */
 /* a8  Weighted combine  [P1 §Drift og omkostninger; P4 §Parallelism/EP]     */
 /* ------------------------------------------------------------------------ */

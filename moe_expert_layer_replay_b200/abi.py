@@ -22,6 +22,7 @@ EXPORTS = [
     "moe_quant_fp8_block", "moe_quant_weights", "moe_grouped_gemm_fp8", "moe_combine",
     "moe_combine_bwd", "moe_unpermute_reduce", "moe_permute_noalloc", "moe_kernel_launches",
     "moe_router_fwd", "moe_capture_payload", "moe_router_bwd_workspace_size", "moe_router_bwd",
+    "moe_grouped_gemm_fp8_seg",
 ]
 
 
@@ -76,6 +77,7 @@ def lib() -> ctypes.CDLL:
             "moe_quant_fp8_block": (ctypes.c_int, [P, I64, I64, I64, I32, I32, P, P, P, P, P]),
             "moe_quant_weights": (ctypes.c_int, [P, P, P, D, P, P, P, P, P, P, P, P, P]),
             "moe_grouped_gemm_fp8": (ctypes.c_int, [I32, D, P, ctypes.POINTER(GemmArgs), P]),
+            "moe_grouped_gemm_fp8_seg": (ctypes.c_int, [I32, D, I64, P, I32, ctypes.POINTER(GemmArgs), P]),
             "moe_combine": (ctypes.c_int, [P, P, P, D, P, P]),
             "moe_combine_bwd": (ctypes.c_int, [P, P, P, P, P, P, P, D, P, P, P, P, P, P]),
             "moe_unpermute_reduce": (ctypes.c_int, [P, P, D, P, P]),
@@ -197,6 +199,15 @@ def grouped_gemm_fp8(op, d: Dims, offsets, a, sa, b, sb, aux=None, out_q=None, o
     g = GemmArgs(*[None if t is None else t.data_ptr() for t in (a, sa, b, sb, aux, out_q, out_s, out_bf16, out_f32)])
     _check("moe_grouped_gemm_fp8", lib().moe_grouped_gemm_fp8(int(op), ctypes.byref(d), _p(offsets),
                                                               ctypes.byref(g), _s(stream)))
+
+
+def grouped_gemm_fp8_seg(op, d: Dims, rows_cap, offsets, n_seg, a, sa, b, sb, aux=None, out_q=None, out_s=None,
+                         out_bf16=None, stream=None):
+    """Grouped GEMM over n_seg row segments; segment v uses expert v % d.E's weights."""
+    g = GemmArgs(*[None if t is None else t.data_ptr() for t in (a, sa, b, sb, aux, out_q, out_s, out_bf16, None)])
+    _check("moe_grouped_gemm_fp8_seg", lib().moe_grouped_gemm_fp8_seg(int(op), ctypes.byref(d), int(rows_cap),
+                                                                      _p(offsets), int(n_seg), ctypes.byref(g),
+                                                                      _s(stream)))
 
 
 def combine(Y, w, pos, d: Dims, y, stream=None):

@@ -84,7 +84,8 @@ static_assert(smem_bytes<EPI_SILU>() <= 232448 && smem_bytes<EPI_BF16>() <= 2324
 
 struct Args {
     const int32_t *offsets;
-    int E;
+    int E;   // row segments (rows mode) or experts (wgrad mode)
+    int ew;  // rows mode: segment v uses the weights of expert v % ew
     int64_t R_cap;
     int M;  // wgrad: rows of dW (D or 2I)
     int N;  // output columns
@@ -160,7 +161,7 @@ __device__ __forceinline__ Tile tile_of(int t, const Args &p, const int *offs_s)
             int mid = (lo + hi + 1) >> 1;
             if (offs_s[mid] <= x.m0) lo = mid; else hi = mid - 1;
         }
-        x.e = lo;
+        x.e = lo < p.ew ? lo : lo % p.ew;   // the weights' expert
         x.kb0 = 0;
         x.kb1 = p.K / BK;
     }
@@ -632,12 +633,13 @@ static int launch_one(const CUtensorMap &a, const CUtensorMap &b, const CUtensor
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
-int launch_grouped_gemm(int op, const moe_dims &d, int64_t R_cap, const int32_t *offsets, const moe_gemm_args &g,
-                        int *status, uint64_t budget, cudaStream_t s)
+int launch_grouped_gemm(int op, const moe_dims &d, int64_t R_cap, const int32_t *offsets, int n_seg,
+                        const moe_gemm_args &g, int *status, uint64_t budget, cudaStream_t s)
 {
     gemm::Args a{};
     a.offsets = offsets;
-    a.E = d.E;
+    a.E = n_seg;
+    a.ew = d.E;
     a.R_cap = R_cap;
     a.sa = g.sa;
     a.sb = g.sb;

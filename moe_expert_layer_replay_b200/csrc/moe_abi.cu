@@ -8,7 +8,7 @@
 #include "common.cuh"
 
 namespace moe {
-int launch_grouped_gemm(int op, const moe_dims &d, int64_t R_cap, const int32_t *offsets,
+int launch_grouped_gemm(int op, const moe_dims &d, int64_t R_cap, const int32_t *offsets, int n_seg,
                         const moe_gemm_args &g, int *status, uint64_t budget, cudaStream_t s);
 }
 
@@ -257,12 +257,10 @@ int moe_quant_weights(const uint16_t *w_gate, const uint16_t *w_up, const uint16
                                      I * D, wdT_s, nD, nI * nD, s);
 }
 
-int moe_grouped_gemm_fp8(int32_t op, const moe_dims *d, const int32_t *offsets, const moe_gemm_args *g,
-                         void *stream)
+namespace {
+int check_gemm_args(int32_t op, const moe_gemm_args *g)
 {
-    int st = check_dims(d, true);
-    if (st) return st;
-    if (!offsets || !g || !g->a || !g->sa || !g->b || !g->sb) return MOE_ERR_INVALID_ARG;
+    if (!g || !g->a || !g->sa || !g->b || !g->sb) return MOE_ERR_INVALID_ARG;
     if (!aligned16(g->a) || !aligned16(g->b)) return MOE_ERR_INVALID_ARG;
     switch (op) {
     case MOE_GEMM_GATEUP_SILU:
@@ -286,10 +284,39 @@ int moe_grouped_gemm_fp8(int32_t op, const moe_dims *d, const int32_t *offsets, 
     default:
         return MOE_ERR_INVALID_ARG;
     }
+    return MOE_OK;
+}
+}  // namespace
+
+int moe_grouped_gemm_fp8(int32_t op, const moe_dims *d, const int32_t *offsets, const moe_gemm_args *g,
+                         void *stream)
+{
+    int st = check_dims(d, true);
+    if (st) return st;
+    if (!offsets) return MOE_ERR_INVALID_ARG;
+    st = check_gemm_args(op, g);
+    if (st) return st;
     int *sp = status_ptr();
     if (!sp) return MOE_ERR_CUDA;
-    return moe::launch_grouped_gemm(op, *d, moe_rows_capacity(d), offsets, *g, sp, wait_budget(),
+    return moe::launch_grouped_gemm(op, *d, moe_rows_capacity(d), offsets, d->E, *g, sp, wait_budget(),
                                     as_stream(stream));
+}
+
+int moe_grouped_gemm_fp8_seg(int32_t op, const moe_dims *d, int64_t rows_cap, const int32_t *offsets, int32_t n_seg,
+                             const moe_gemm_args *g, void *stream)
+{
+    int st = check_dims(d, true);
+    if (st) return st;
+    if (op != MOE_GEMM_GATEUP_SILU && op != MOE_GEMM_DOWN && op != MOE_GEMM_DGRAD_DOWN_SILU &&
+        op != MOE_GEMM_DGRAD_GATEUP)
+        return MOE_ERR_INVALID_ARG;
+    if (!offsets || rows_cap < 0 || rows_cap % 128 || n_seg <= 0 || n_seg > 256 || n_seg % d->E)
+        return MOE_ERR_INVALID_ARG;
+    st = check_gemm_args(op, g);
+    if (st) return st;
+    int *sp = status_ptr();
+    if (!sp) return MOE_ERR_CUDA;
+    return moe::launch_grouped_gemm(op, *d, rows_cap, offsets, n_seg, *g, sp, wait_budget(), as_stream(stream));
 }
 
 int moe_combine(const uint16_t *Y, const float *w, const int32_t *pos, const moe_dims *d, uint16_t *y,
