@@ -272,6 +272,19 @@ typedef struct {
 int moe_grouped_gemm_fp8(int32_t op, const moe_dims *dims, const int32_t *offsets,
                          const moe_gemm_args *args, void *stream);
 
+/* a4+a6 without the permuted copy of the activations: GATEUP_SILU whose A
+ * operand is gathered from the token rows by the GEMM's loads (TMA
+ * tile::gather4), so the dispatch writes no R x D FP8 copy.  args->a =
+ * codes [T][D] and args->sa = scales [D/128][T] of the 1x128 quantisation of
+ * x itself (moe_quant_fp8_block(x, T, D, D, 1, 128, ...)); permuted row r
+ * is token src_idx[r] / k (src_idx from moe_permute), a row with src_idx < 0
+ * is zero.  Every other operand and every output is that of GATEUP_SILU, so
+ * the results equal those of moe_permute's dispatch followed by
+ * moe_grouped_gemm_fp8(GATEUP_SILU) [P1 §Drift og omkostninger: the
+ * dispatch/combine cost of every layer]. */
+int moe_gateup_gather_fp8(const moe_dims *dims, const int32_t *offsets, const int32_t *src_idx,
+                          const moe_gemm_args *args, void *stream);
+
 /* The same GEMMs (rows-mode ops only: GATEUP_SILU, DOWN, DGRAD_DOWN_SILU,
  * DGRAD_GATEUP) over n_seg 128-aligned row segments offsets[0..n_seg] that
  * are not one per expert: segment v uses the weights of expert v % dims->E

@@ -22,7 +22,7 @@ EXPORTS = [
     "moe_quant_fp8_block", "moe_quant_weights", "moe_grouped_gemm_fp8", "moe_combine",
     "moe_combine_bwd", "moe_unpermute_reduce", "moe_permute_noalloc", "moe_kernel_launches",
     "moe_router_fwd", "moe_capture_payload", "moe_router_bwd_workspace_size", "moe_router_bwd",
-    "moe_grouped_gemm_fp8_seg",
+    "moe_grouped_gemm_fp8_seg", "moe_gateup_gather_fp8",
 ]
 
 
@@ -78,6 +78,7 @@ def lib() -> ctypes.CDLL:
             "moe_quant_weights": (ctypes.c_int, [P, P, P, D, P, P, P, P, P, P, P, P, P]),
             "moe_grouped_gemm_fp8": (ctypes.c_int, [I32, D, P, ctypes.POINTER(GemmArgs), P]),
             "moe_grouped_gemm_fp8_seg": (ctypes.c_int, [I32, D, I64, P, I32, ctypes.POINTER(GemmArgs), P]),
+            "moe_gateup_gather_fp8": (ctypes.c_int, [D, P, P, ctypes.POINTER(GemmArgs), P]),
             "moe_combine": (ctypes.c_int, [P, P, P, D, P, P]),
             "moe_combine_bwd": (ctypes.c_int, [P, P, P, P, P, P, P, D, P, P, P, P, P, P]),
             "moe_unpermute_reduce": (ctypes.c_int, [P, P, D, P, P]),
@@ -208,6 +209,15 @@ def grouped_gemm_fp8_seg(op, d: Dims, rows_cap, offsets, n_seg, a, sa, b, sb, au
     _check("moe_grouped_gemm_fp8_seg", lib().moe_grouped_gemm_fp8_seg(int(op), ctypes.byref(d), int(rows_cap),
                                                                       _p(offsets), int(n_seg), ctypes.byref(g),
                                                                       _s(stream)))
+
+
+def gateup_gather_fp8(d: Dims, offsets, src_idx, a_tok, sa_tok, b, sb, aux=None, out_q=None, out_s=None,
+                      out_bf16=None, stream=None):
+    """GATEUP_SILU with A gathered from the token-row codes (no permuted copy)."""
+    g = GemmArgs(*[None if t is None else t.data_ptr() for t in (a_tok, sa_tok, b, sb, aux, out_q, out_s, out_bf16,
+                                                                None)])
+    _check("moe_gateup_gather_fp8", lib().moe_gateup_gather_fp8(ctypes.byref(d), _p(offsets), _p(src_idx),
+                                                                ctypes.byref(g), _s(stream)))
 
 
 def combine(Y, w, pos, d: Dims, y, stream=None):

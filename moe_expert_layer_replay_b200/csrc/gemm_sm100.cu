@@ -99,6 +99,12 @@ struct Args {
     float *out_f32;
     int *status;
     uint64_t budget;
+    // gather (a6 only): A rows come from the token-row codes, row r of the
+    // permuted layout being token src_idx[r] / k (no row for src_idx < 0);
+    // row scales sa[kb * T + token]
+    const int32_t *src_idx;
+    int k;
+    int T;
 };
 
 // ----------------------------------------------------------------- PTX ----
@@ -116,6 +122,19 @@ __device__ __forceinline__ void mma_f8(uint32_t tmem_d, uint64_t a, uint64_t b, 
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
         "l"(a), "l"(b), "r"(IDESC), "r"(accum));
+}
+
+// Four rows (row coordinates r0..r3, the same 128-byte column window c0) of a
+// tensor whose map has a one-row box, into four consecutive 128-byte rows of
+// shared memory.
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap *map, int32_t c0, int32_t r0,
+                                            int32_t r1, int32_t r2, int32_t r3, uint32_t bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+        : "memory");
 }
 
 // ------------------------------------------------------------ schedule ----
@@ -169,7 +188,7 @@ __device__ __forceinline__ Tile tile_of(int t, const Args &p, const int *offs_s)
 }
 
 // --------------------------------------------------------------- kernel ----
-template <int kEpi>
+template <int kEpi, bool kGather = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmC, const Args p)
@@ -228,7 +247,48 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 
     if (warp < EPI_WARP0) {
       asm volatile("setmaxnreg.dec.sync.aligned.u32 56;");
-      if (warp == 0) {
+      if (warp == 0 && kGather) {
+        // ------------------------------------- TMA producer, gathering ----
+        // every lane gathers four A rows (tile rows 4*lane .. 4*lane+3) of
+        // each K block from the token-row codes; lane 0 also loads B
+        int stage = 0;
+        uint32_t phase = 0;
+        uint32_t pend = 0, pend_phase = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+            const Tile x = tile_of<false>(t, p, offs_s);
+            int tok[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int si = p.src_idx[x.m0 + 4 * lane + i];
+                tok[i] = si >= 0 ? si / p.k : p.T;   // row T is out of range: zeros
+            }
+            for (int kb = x.kb0; kb < x.kb1; ++kb) {
+                if (!warp_wait_bounded(bar_empty + 8 * stage, phase ^ 1, p.budget, abort_flag, p.status)) {
+                    ok = false;
+                    break;
+                }
+                pend &= ~(1u << stage);
+                const uint32_t fb = bar_full + 8 * stage;
+                const uint32_t dA = sbase + stage * STAGE_BYTES, dB = dA + A_BYTES;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(fb, STAGE_BYTES);
+                    tma_load_2d(dB, &tmB, kb * BK, x.e * p.N + x.n0, fb);
+                }
+                __syncwarp();
+                tma_gather4(dA + 512 * lane, &tmA, kb * BK, tok[0], tok[1], tok[2], tok[3], fb);
+                pend |= 1u << stage;
+                pend_phase = (pend_phase & ~(1u << stage)) | (phase << stage);
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1;
+                }
+            }
+        }
+        if (!ok && lane == 0)
+            for (int s = 0; s < STAGES; ++s)
+                if (pend & (1u << s)) wait_drain(bar_full + 8 * s, (pend_phase >> s) & 1u);
+      } else if (warp == 0) {
         // ------------------------------------------------ TMA producer ----
         if (lane == 0) {
             int stage = 0;
@@ -365,8 +425,16 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             // into registers (row scale, weight-block scale(s)).  Wgrad: the
             // producer bulk-copies them into the scale ring, up to SC_SLOTS K
             // blocks ahead; each warp releases a slot after reading it.
+            int tok_r = 0;
+            if (kGather) {
+                const int si = p.src_idx[x.m0 + row];
+                tok_r = si >= 0 ? si / p.k : -1;
+            }
             auto load_rows = [&](int kb, float &a, float &b0, float &b1) {
-                a = p.sa[(int64_t)kb * p.R_cap + x.m0 + row];
+                if (kGather)
+                    a = tok_r >= 0 ? p.sa[(int64_t)kb * p.T + tok_r] : 0.0f;
+                else
+                    a = p.sa[(int64_t)kb * p.R_cap + x.m0 + row];
                 const int64_t sbrow = (int64_t)x.e * NB + 2 * x.nt;
                 if (kEpi == EPI_SILU) {
                     b0 = p.sb[sbrow * KB + kb];        // gate block
@@ -617,18 +685,18 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 // ------------------------------------------------------------------ host ----
 using namespace sm100;
 
-template <int kEpi>
+template <int kEpi, bool kGather = false>
 static int launch_one(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &c, const gemm::Args &args,
                       int grid, cudaStream_t s)
 {
     static bool configured = false;  // per process; attribute is per function
     if (!configured) {
-        if (cudaFuncSetAttribute(gemm::grouped_gemm_kernel<kEpi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(gemm::grouped_gemm_kernel<kEpi, kGather>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  gemm::smem_bytes<kEpi>()) != cudaSuccess)
             return MOE_ERR_CUDA;
         configured = true;
     }
-    gemm::grouped_gemm_kernel<kEpi><<<grid, gemm::NUM_THREADS, gemm::smem_bytes<kEpi>(), s>>>(a, b, c, args);
+    gemm::grouped_gemm_kernel<kEpi, kGather><<<grid, gemm::NUM_THREADS, gemm::smem_bytes<kEpi>(), s>>>(a, b, c, args);
     count_launch();
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
@@ -694,6 +762,38 @@ int launch_grouped_gemm(int op, const moe_dims &d, int64_t R_cap, const int32_t 
     case MOE_GEMM_DGRAD_DOWN_SILU: return launch_one<gemm::EPI_DSILU>(mA, mB, mC, a, grid, s);
     default: return launch_one<gemm::EPI_WGRAD>(mA, mB, mC, a, grid, s);
     }
+}
+
+// a6 with its A operand gathered from the token rows: codes xq_tok [T][D]
+// (g.a) and 1x128 scales [D/128][T] (g.sa); permuted row r is token
+// src_idx[r] / k.  The tensor map has one-row boxes (tile::gather4).
+int launch_gateup_gather(const moe_dims &d, int64_t R_cap, const int32_t *offsets, const int32_t *src_idx,
+                         const moe_gemm_args &g, int *status, uint64_t budget, cudaStream_t s)
+{
+    gemm::Args a{};
+    a.offsets = offsets;
+    a.E = d.E;
+    a.ew = d.E;
+    a.R_cap = R_cap;
+    a.sa = g.sa;
+    a.sb = g.sb;
+    a.aux = g.aux;
+    a.out_q = g.out_q;
+    a.out_s = g.out_s;
+    a.out_bf16 = g.out_bf16;
+    a.status = status;
+    a.budget = budget;
+    a.src_idx = src_idx;
+    a.k = d.k;
+    a.T = d.T;
+    const int64_t D = d.D, I = d.I, E = d.E;
+    a.N = (int)(2 * I);
+    a.K = (int)D;
+    CUtensorMap mA, mB, mC;
+    if (!make_map(&mA, g.a, D, d.T, 1) || !make_map(&mB, g.b, D, E * 2 * I, 256) ||
+        !make_store_map(&mC, g.out_q, I, R_cap, 1))
+        return MOE_ERR_CUDA;
+    return launch_one<gemm::EPI_SILU, true>(mA, mB, mC, a, sm_count(), s);
 }
 
 }  // namespace moe

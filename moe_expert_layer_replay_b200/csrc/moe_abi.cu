@@ -10,6 +10,8 @@
 namespace moe {
 int launch_grouped_gemm(int op, const moe_dims &d, int64_t R_cap, const int32_t *offsets, int n_seg,
                         const moe_gemm_args &g, int *status, uint64_t budget, cudaStream_t s);
+int launch_gateup_gather(const moe_dims &d, int64_t R_cap, const int32_t *offsets, const int32_t *src_idx,
+                         const moe_gemm_args &g, int *status, uint64_t budget, cudaStream_t s);
 }
 
 // Latched device status word (one per device that loads the library).
@@ -300,6 +302,21 @@ int moe_grouped_gemm_fp8(int32_t op, const moe_dims *d, const int32_t *offsets, 
     if (!sp) return MOE_ERR_CUDA;
     return moe::launch_grouped_gemm(op, *d, moe_rows_capacity(d), offsets, d->E, *g, sp, wait_budget(),
                                     as_stream(stream));
+}
+
+int moe_gateup_gather_fp8(const moe_dims *d, const int32_t *offsets, const int32_t *src_idx,
+                          const moe_gemm_args *g, void *stream)
+{
+    int st = check_dims(d, true);
+    if (st) return st;
+    if (!offsets || !src_idx) return MOE_ERR_INVALID_ARG;
+    st = check_gemm_args(MOE_GEMM_GATEUP_SILU, g);
+    if (st) return st;
+    if (d->T == 0) return MOE_OK;   // no token: every segment is empty
+    int *sp = status_ptr();
+    if (!sp) return MOE_ERR_CUDA;
+    return moe::launch_gateup_gather(*d, moe_rows_capacity(d), offsets, src_idx, *g, sp, wait_budget(),
+                                     as_stream(stream));
 }
 
 int moe_grouped_gemm_fp8_seg(int32_t op, const moe_dims *d, int64_t rows_cap, const int32_t *offsets, int32_t n_seg,
