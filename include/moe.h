@@ -91,6 +91,14 @@ void moe_set_wait_budget(uint64_t cycles);
  * again without calling into the library).  For accounting only. */
 uint64_t moe_kernel_launches(void);
 
+/* Which kernel runs the rows-mode grouped GEMMs (GATEUP_SILU, DOWN,
+ * DGRAD_DOWN_SILU, DGRAD_GATEUP): 0 = one SM per 128 x 256 tile (the
+ * default), 1 = the 2-SM MMA (a pair of SMs per 256 x 256 tile, each loading
+ * half of the weight tile), -1 = chosen per call from the shapes.  Results
+ * are the same bit for bit; the choice is per process.  Returns
+ * MOE_ERR_INVALID_ARG for any other value. */
+int moe_set_gemm_variant(int variant);
+
 /* ------------------------------------------------------------------------ */
 /* a1  Top-k routing  [P1 §Drift og omkostninger i realiteten]               */
 /* ------------------------------------------------------------------------ */

@@ -22,7 +22,7 @@ EXPORTS = [
     "moe_quant_fp8_block", "moe_quant_weights", "moe_grouped_gemm_fp8", "moe_combine",
     "moe_combine_bwd", "moe_unpermute_reduce", "moe_permute_noalloc", "moe_kernel_launches",
     "moe_router_fwd", "moe_capture_payload", "moe_router_bwd_workspace_size", "moe_router_bwd",
-    "moe_grouped_gemm_fp8_seg", "moe_gateup_gather_fp8",
+    "moe_grouped_gemm_fp8_seg", "moe_gateup_gather_fp8", "moe_set_gemm_variant",
 ]
 
 
@@ -66,6 +66,7 @@ def lib() -> ctypes.CDLL:
             "moe_get_status": (ctypes.c_int, [P, ctypes.POINTER(ctypes.c_int)]),
             "moe_set_wait_budget": (None, [U64]),
             "moe_kernel_launches": (U64, []),
+            "moe_set_gemm_variant": (ctypes.c_int, [ctypes.c_int]),
             "moe_route_topk": (ctypes.c_int, [P, D, P, P, P]),
             "moe_route_replay": (ctypes.c_int, [P, I32, I32, D, P, P, P, P, P]),
             "moe_router_fwd": (ctypes.c_int, [P, P, D, P, P, P, P]),
@@ -135,6 +136,11 @@ def get_status(stream=None) -> int:
 
 def set_wait_budget(cycles: int) -> None:
     lib().moe_set_wait_budget(int(cycles))
+
+
+def set_gemm_variant(variant: int) -> None:
+    """0: one-SM tiles (default), 1: the 2-SM MMA, -1: chosen per call."""
+    _check("moe_set_gemm_variant", lib().moe_set_gemm_variant(int(variant)))
 
 
 def kernel_launches() -> int:

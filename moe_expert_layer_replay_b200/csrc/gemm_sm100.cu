@@ -38,15 +38,21 @@ namespace moe {
 namespace gemm {
 
 constexpr int BM = 128, BN = 256, BK = 128;
-constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * BK, B_BYTES = BN * BK, STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int A_BYTES = BM * BK;
 constexpr int NUM_THREADS = 384;
 constexpr int EPI_WARP0 = 4;
 constexpr int EPI_THREADS = 256;
 constexpr uint32_t TMEM_COLS = 512;
-// smem: operand ring | barriers (full[4], empty[4], tfull[2], tempty[2], drain, epi) |
-// tmem slot | abort flag | offsets[257] | then, 1024-aligned, a region whose
-// use depends on the epilogue:
+constexpr int WS_FLOATS = 128 + 256;
+constexpr int SC_SLOTS = 8;
+constexpr int TSTORE_BUF = 32 * 64;
+
+// Shared memory of one variant (kPair: the 2-SM MMA, where each CTA of a pair
+// holds its own 128 rows of A and half of B):
+//   operand ring [STAGES][A tile | B tile] | barriers (full[STAGES],
+//   empty[STAGES], tfull[2], tempty[2], drain, epi) | tmem slot | abort flag |
+//   offsets[257] | (kPair) pair-tile prefix sums[257] | then, 1024-aligned, a
+//   region whose use depends on the epilogue:
 //   SILU   amax exchange [2][2][128] fp32 | h-code store buffers [8 warps][32 rows][64 B]
 //   BF16   output store buffers [8 warps][2][32 rows][64 B]
 //   WGRAD  scale ring [SC_SLOTS][128 row + 256 column] fp32 with its own
@@ -54,33 +60,41 @@ constexpr uint32_t TMEM_COLS = 512;
 //          epilogue warps), deeper than the operand ring
 //   DSILU  unused
 // Store buffers are read by TMA stores (32 rows x 64 bytes boxes, no swizzle).
-constexpr int OFF_BAR = STAGES * STAGE_BYTES;
-constexpr int OFF_TMEM_SLOT = OFF_BAR + 16 * 8;
-constexpr int OFF_ABORT = OFF_TMEM_SLOT + 4;
-constexpr int OFF_OFFSETS = OFF_BAR + 256;
-constexpr int OFF_EPI = (OFF_OFFSETS + 1040 + 1023) / 1024 * 1024;
-constexpr int OFF_AMAX = OFF_EPI;
-constexpr int OFF_WS = OFF_EPI;
-constexpr int WS_FLOATS = 128 + 256;
-constexpr int SC_SLOTS = 8;
-constexpr int OFF_WS_BAR = OFF_WS + SC_SLOTS * WS_FLOATS * 4;  // sfull[SC_SLOTS], sempty[SC_SLOTS]
-constexpr int TSTORE_BUF = 32 * 64;
-constexpr int OFF_TSTORE_SILU = OFF_EPI + 2 * 2 * 128 * 4;
-constexpr int OFF_TSTORE_BF16 = OFF_EPI;
+template <bool kPair>
+struct Lay {
+    static constexpr int STAGES = kPair ? 5 : 4;
+    static constexpr int B_BYTES = (kPair ? BN / 2 : BN) * BK;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int OFF_BAR = STAGES * STAGE_BYTES;
+    static constexpr int OFF_TMEM_SLOT = OFF_BAR + 24 * 8;
+    static constexpr int OFF_ABORT = OFF_TMEM_SLOT + 4;
+    static constexpr int OFF_OFFSETS = OFF_BAR + 256;
+    static constexpr int OFF_PAIRS = OFF_OFFSETS + 1040;
+    static constexpr int OFF_EPI = (OFF_PAIRS + (kPair ? 1040 : 0) + 1023) / 1024 * 1024;
+    static constexpr int OFF_AMAX = OFF_EPI;
+    static constexpr int OFF_WS = OFF_EPI;
+    static constexpr int OFF_WS_BAR = OFF_WS + SC_SLOTS * WS_FLOATS * 4;  // sfull[SC_SLOTS], sempty[SC_SLOTS]
+    static constexpr int OFF_TSTORE_SILU = OFF_EPI + 2 * 2 * 128 * 4;
+    static constexpr int OFF_TSTORE_BF16 = OFF_EPI;
+};
 
 enum Epi { EPI_SILU = 0, EPI_BF16 = 1, EPI_DSILU = 2, EPI_WGRAD = 3 };
 
-template <int kEpi>
+template <int kEpi, bool kPair = false>
 constexpr int smem_bytes()
 {
-    return 1024 + (kEpi == EPI_SILU   ? OFF_TSTORE_SILU + 8 * TSTORE_BUF
-                   : kEpi == EPI_BF16 ? OFF_TSTORE_BF16 + 8 * 2 * TSTORE_BUF
-                   : kEpi == EPI_WGRAD ? OFF_WS_BAR + 2 * SC_SLOTS * 8
-                                       : OFF_EPI);  // + alignment slack
+    using L = Lay<kPair>;
+    return 1024 + (kEpi == EPI_SILU   ? L::OFF_TSTORE_SILU + 8 * TSTORE_BUF
+                   : kEpi == EPI_BF16 ? L::OFF_TSTORE_BF16 + 8 * 2 * TSTORE_BUF
+                   : kEpi == EPI_WGRAD ? L::OFF_WS_BAR + 2 * SC_SLOTS * 8
+                                       : L::OFF_EPI);  // + alignment slack
 }
 static_assert(smem_bytes<EPI_SILU>() <= 232448 && smem_bytes<EPI_BF16>() <= 232448 &&
-                  smem_bytes<EPI_WGRAD>() <= 232448 && smem_bytes<EPI_DSILU>() <= 232448,
+                  smem_bytes<EPI_WGRAD>() <= 232448 && smem_bytes<EPI_DSILU>() <= 232448 &&
+                  smem_bytes<EPI_SILU, true>() <= 232448 && smem_bytes<EPI_BF16, true>() <= 232448 &&
+                  smem_bytes<EPI_DSILU, true>() <= 232448,
               "shared memory budget");
+static_assert(Lay<false>::OFF_EPI == 198656, "the one-SM layout is unchanged");
 
 struct Args {
     const int32_t *offsets;
@@ -124,6 +138,71 @@ __device__ __forceinline__ void mma_f8(uint32_t tmem_d, uint64_t a, uint64_t b, 
         "l"(a), "l"(b), "r"(IDESC), "r"(accum));
 }
 
+// The 2-SM MMA (cta_group::2): M = 256 over the CTA pair (128 rows of A in
+// each CTA's shared memory at the same offset), N = 256 (each CTA holds 128
+// rows of B: the leader rows 0-127, the peer rows 128-255), D in each CTA's
+// TMEM (its own 128 rows).  Issued by the leader CTA only.
+constexpr uint32_t IDESC_PAIR = (1u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                                ((uint32_t)(2 * BM >> 4) << 24);
+
+__device__ __forceinline__ void mma_f8_pair(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t accum)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(a), "l"(b), "r"(IDESC_PAIR), "r"(accum));
+}
+
+// Arrives once, when the leader's MMAs issued so far are done, on the barrier
+// at this offset in each CTA of the pair.
+__device__ __forceinline__ void mma_commit_pair(uint32_t bar)
+{
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+        "h"((uint16_t)3)
+        : "memory");
+}
+
+__device__ __forceinline__ uint32_t cluster_rank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// shared::cluster address of the same shared-memory offset in CTA `rank`
+__device__ __forceinline__ uint32_t peer_addr(uint32_t a, uint32_t rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync_all()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// arrive on an mbarrier given by its shared::cluster address (any CTA of the cluster)
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+// TMA tile load into this CTA's shared memory whose completion is counted on
+// an mbarrier of either CTA of the pair (shared::cluster address).  No
+// multicast: every CTA loads its own bytes.
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap *map, int32_t c0, int32_t c1,
+                                                 uint32_t bar_cluster)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1)
+        : "memory");
+}
+
 // Four rows (row coordinates r0..r3, the same 128-byte column window c0) of a
 // tensor whose map has a one-row box, into four consecutive 128-byte rows of
 // shared memory.
@@ -145,21 +224,27 @@ struct Tile {
     int nt;     // column-tile index
     int kb0;    // first K block
     int kb1;    // one past the last K block
+    bool valid; // this CTA's rows belong to the tile (a pair's second half may not)
 };
 
-template <bool kWgrad>
-__device__ __forceinline__ int num_tiles(const Args &p, const int *offs_s)
+// Pair mode: segment v of 128-row tiles mt_v = (offs[v+1] - offs[v]) / 128 has
+// ceil(mt_v / 2) pair tiles; pps[v] counts them before segment v.
+template <bool kWgrad, bool kPair>
+__device__ __forceinline__ int num_tiles(const Args &p, const int *offs_s, const int *pps_s)
 {
     const int NT = (p.N + BN - 1) / BN;
     if (kWgrad) return p.E * (p.M / BM) * NT;
+    if (kPair) return pps_s[p.E] * NT;
     return (offs_s[p.E] / BM) * NT;
 }
 
-template <bool kWgrad>
-__device__ __forceinline__ Tile tile_of(int t, const Args &p, const int *offs_s)
+template <bool kWgrad, bool kPair = false>
+__device__ __forceinline__ Tile tile_of(int t, const Args &p, const int *offs_s, const int *pps_s = nullptr,
+                                        uint32_t rank = 0)
 {
     const int NT = (p.N + BN - 1) / BN;
     Tile x;
+    x.valid = true;
     if (kWgrad) {
         const int MT = p.M / BM;
         x.e = t / (MT * NT);
@@ -170,6 +255,21 @@ __device__ __forceinline__ Tile tile_of(int t, const Args &p, const int *offs_s)
         x.n0 = x.nt * BN;
         x.kb0 = offs_s[x.e] / BK;
         x.kb1 = offs_s[x.e + 1] / BK;
+    } else if (kPair) {
+        const int pt = t / NT;
+        x.nt = t - pt * NT;
+        x.n0 = x.nt * BN;
+        int lo = 0, hi = p.E - 1;  // last v with pps[v] <= pt
+        while (lo < hi) {
+            int mid = (lo + hi + 1) >> 1;
+            if (pps_s[mid] <= pt) lo = mid; else hi = mid - 1;
+        }
+        const int base = offs_s[lo] + 2 * BM * (pt - pps_s[lo]);
+        x.m0 = base + BM * (int)rank;
+        x.valid = x.m0 < offs_s[lo + 1];
+        x.e = lo < p.ew ? lo : lo % p.ew;
+        x.kb0 = 0;
+        x.kb1 = p.K / BK;
     } else {
         int mt = t / NT;
         x.nt = t - mt * NT;
@@ -188,12 +288,19 @@ __device__ __forceinline__ Tile tile_of(int t, const Args &p, const int *offs_s)
 }
 
 // --------------------------------------------------------------- kernel ----
-template <int kEpi, bool kGather = false>
+template <int kEpi, bool kGather = false, bool kPair = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmC, const Args p)
 {
     constexpr bool kWgrad = (kEpi == EPI_WGRAD);
+    static_assert(!(kPair && (kWgrad || kGather)), "the 2-SM variant covers the rows-mode GEMMs");
+    using L = Lay<kPair>;
+    constexpr int STAGES = L::STAGES, STAGE_BYTES = L::STAGE_BYTES;
+    constexpr int OFF_BAR = L::OFF_BAR, OFF_ABORT = L::OFF_ABORT, OFF_TMEM_SLOT = L::OFF_TMEM_SLOT;
+    constexpr int OFF_OFFSETS = L::OFF_OFFSETS, OFF_AMAX = L::OFF_AMAX, OFF_WS = L::OFF_WS;
+    constexpr int OFF_WS_BAR = L::OFF_WS_BAR, OFF_TSTORE_SILU = L::OFF_TSTORE_SILU;
+    constexpr int OFF_TSTORE_BF16 = L::OFF_TSTORE_BF16;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const uint32_t sbase = smem_u32(smem);
@@ -206,14 +313,32 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_ABORT);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_TMEM_SLOT);
     int *offs_s = reinterpret_cast<int *>(smem + OFF_OFFSETS);
+    int *pps_s = reinterpret_cast<int *>(smem + L::OFF_PAIRS);        // pair mode: [E+1]
     float *amax_s = reinterpret_cast<float *>(smem + OFF_AMAX);       // [2][2][128]
     float *wscale = reinterpret_cast<float *>(smem + OFF_WS);          // wgrad: [SC_SLOTS][WS_FLOATS]
     const uint32_t bar_sfull = sbase + OFF_WS_BAR;                     // wgrad: [SC_SLOTS]
     const uint32_t bar_sempty = bar_sfull + SC_SLOTS * 8;              // wgrad: [SC_SLOTS]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // pair mode: CTA `rank` of the pair (0 leads: it issues the MMAs and
+    // holds the barriers the pair's loads and TMEM releases count on); the
+    // pairs walk the tiles together
+    const uint32_t rank = kPair ? cluster_rank() : 0;
+    const int t_first = kPair ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+    const int t_step = kPair ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
     for (int i = threadIdx.x; i <= p.E; i += blockDim.x) offs_s[i] = p.offsets[i];
+    if (kPair) {
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            int acc = 0;
+            for (int v = 0; v < p.E; ++v) {
+                pps_s[v] = acc;
+                acc += ((offs_s[v + 1] - offs_s[v]) / BM + 1) / 2;
+            }
+            pps_s[p.E] = acc;
+        }
+    }
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(bar_full + 8 * s, 1);
@@ -226,7 +351,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             }
         for (int b = 0; b < 2; ++b) {
             mbar_init(bar_tfull + 8 * b, 1);
-            mbar_init(bar_tempty + 8 * b, EPI_THREADS / 32);
+            mbar_init(bar_tempty + 8 * b, (kPair ? 2 : 1) * EPI_THREADS / 32);
         }
         mbar_init(bar_drain, 1);
         mbar_init(bar_epi, EPI_THREADS);
@@ -235,15 +360,25 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
     if (warp == 1) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                     "r"(TMEM_COLS));
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+        if (kPair) {
+            asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                         "r"(TMEM_COLS));
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+        } else {
+            asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                         "r"(TMEM_COLS));
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+        }
     }
     tc_fence_before();
     __syncthreads();
+    if (kPair) cluster_sync_all();   // both CTAs' barriers exist before either signals the other's
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    const int ntiles = num_tiles<kWgrad>(p, offs_s);
+    const int ntiles = num_tiles<kWgrad, kPair>(p, offs_s, pps_s);
+    // the leader's barriers as the pair addresses them
+    const uint32_t lead_full = kPair ? peer_addr(bar_full, 0) : bar_full;
+    const uint32_t lead_tempty = kPair ? peer_addr(bar_tempty, 0) : bar_tempty;
 
     if (warp < EPI_WARP0) {
       asm volatile("setmaxnreg.dec.sync.aligned.u32 56;");
@@ -297,8 +432,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             int sslot = 0;                      // wgrad scale ring
             uint32_t sphase = 0, spend = 0, spend_phase = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-                const Tile x = tile_of<kWgrad>(t, p, offs_s);
+            for (int t = t_first; t < ntiles && ok; t += t_step) {
+                const Tile x = tile_of<kWgrad, kPair>(t, p, offs_s, pps_s, rank);
                 for (int kb = x.kb0; kb < x.kb1; ++kb) {
                     if (!wait_bounded(bar_empty + 8 * stage, phase ^ 1, p.budget, abort_flag, p.status)) {
                         ok = false;
@@ -328,6 +463,13 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                         mbar_arrive_expect_tx(fb, STAGE_BYTES);
                         tma_load_2d(dA, &tmA, kb * BK, x.m0, fb);
                         tma_load_2d(dB, &tmB, kb * BK, x.n0, fb);
+                    } else if (kPair) {
+                        // this CTA's 128 rows of A and 128 rows of B; both CTAs'
+                        // bytes complete on the leader's full barrier
+                        const uint32_t lfb = lead_full + 8 * stage;
+                        if (rank == 0) mbar_arrive_expect_tx(fb, 2 * STAGE_BYTES);
+                        tma_load_2d_pair(dA, &tmA, kb * BK, x.m0, lfb);
+                        tma_load_2d_pair(dB, &tmB, kb * BK, x.e * p.N + x.n0 + (BN / 2) * (int)rank, lfb);
                     } else {
                         mbar_arrive_expect_tx(fb, STAGE_BYTES);
                         tma_load_2d(dA, &tmA, kb * BK, x.m0, fb);
@@ -341,7 +483,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     }
                 }
             }
-            if (!ok) {
+            // (pair mode: the peer's loads complete on the leader's barriers;
+            // the leader's drain waits for the stages it announced, and the
+            // pair leaves together after the closing cluster barrier)
+            if (!ok && rank == 0) {
                 for (int s = 0; s < STAGES; ++s)
                     if (pend & (1u << s)) wait_drain(bar_full + 8 * s, (pend_phase >> s) & 1u);
                 if (kWgrad)
@@ -351,14 +496,15 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         }
     } else if (warp == 1) {
         // ------------------------------------------------- MMA issuer ----
-        if (lane == 0) {
+        // (pair mode: the leader only; its MMAs span both CTAs)
+        if (lane == 0 && rank == 0) {
             int stage = 0;
             uint32_t phase = 0;
             int buf = 0;
             uint32_t bphase = 0;
             bool ok = true, issued = false;
-            for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-                const Tile x = tile_of<kWgrad>(t, p, offs_s);
+            for (int t = t_first; t < ntiles && ok; t += t_step) {
+                const Tile x = tile_of<kWgrad, kPair>(t, p, offs_s, pps_s, rank);
                 for (int kb = x.kb0; kb < x.kb1; ++kb) {
                     if (!wait_bounded(bar_tempty + 8 * buf, bphase ^ 1, p.budget, abort_flag, p.status)) {
                         ok = false;
@@ -372,12 +518,20 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     tc_fence_after();
                     const uint32_t aA = sbase + stage * STAGE_BYTES, aB = aA + A_BYTES;
                     const uint32_t dtm = tmem_base + (uint32_t)(buf * BN);
+                    if (kPair) {
 #pragma unroll
-                    for (int k4 = 0; k4 < BK / 32; ++k4)
-                        mma_f8(dtm, sdesc(aA + 32 * k4), sdesc(aB + 32 * k4), k4 > 0 ? 1u : 0u);
+                        for (int k4 = 0; k4 < BK / 32; ++k4)
+                            mma_f8_pair(dtm, sdesc(aA + 32 * k4), sdesc(aB + 32 * k4), k4 > 0 ? 1u : 0u);
+                        mma_commit_pair(bar_empty + 8 * stage);   // both CTAs' stage is free
+                        mma_commit_pair(bar_tfull + 8 * buf);     // both CTAs' epilogues may read
+                    } else {
+#pragma unroll
+                        for (int k4 = 0; k4 < BK / 32; ++k4)
+                            mma_f8(dtm, sdesc(aA + 32 * k4), sdesc(aB + 32 * k4), k4 > 0 ? 1u : 0u);
+                        mma_commit(bar_empty + 8 * stage);
+                        mma_commit(bar_tfull + 8 * buf);
+                    }
                     issued = true;
-                    mma_commit(bar_empty + 8 * stage);
-                    mma_commit(bar_tfull + 8 * buf);
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1;
@@ -387,7 +541,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 }
             }
             if (issued) {
-                mma_commit(bar_drain);
+                if (kPair)
+                    mma_commit_pair(bar_drain);
+                else
+                    mma_commit(bar_drain);
                 wait_drain(bar_drain, 0);
             }
         }
@@ -415,8 +572,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             ephase ^= 1;
             return r;
         };
-        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++tcount) {
-            const Tile x = tile_of<kWgrad>(t, p, offs_s);
+        for (int t = t_first; t < ntiles && ok; t += t_step, ++tcount) {
+            const Tile x = tile_of<kWgrad, kPair>(t, p, offs_s, pps_s, rank);
             if (kWgrad && x.kb1 == x.kb0) continue;
             float acc[128];
 #pragma unroll
@@ -433,8 +590,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             auto load_rows = [&](int kb, float &a, float &b0, float &b1) {
                 if (kGather)
                     a = tok_r >= 0 ? p.sa[(int64_t)kb * p.T + tok_r] : 0.0f;
-                else
-                    a = p.sa[(int64_t)kb * p.R_cap + x.m0 + row];
+                else   // (a pair's idle half may lie past the last row)
+                    a = x.valid ? p.sa[(int64_t)kb * p.R_cap + x.m0 + row] : 0.0f;
                 const int64_t sbrow = (int64_t)x.e * NB + 2 * x.nt;
                 if (kEpi == EPI_SILU) {
                     b0 = p.sb[sbrow * KB + kb];        // gate block
@@ -444,7 +601,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     b1 = b0;
                 }
             };
-            if (kEpi == EPI_DSILU && (2 * x.nt + h) * 128 < p.N) {
+            if (kEpi == EPI_DSILU && x.valid && (2 * x.nt + h) * 128 < p.N) {
                 // the saved g, u this thread reads after the last K block: to L2 now
                 const uint16_t *gu = p.aux + ((int64_t)x.m0 + row) * 2 * (int64_t)p.N + (int64_t)(2 * x.nt + h) * 256;
 #pragma unroll
@@ -496,7 +653,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                         if (c == 2) {
                             tc_fence_before();
                             __syncwarp();
-                            if (lane == 0) mbar_arrive(bar_tempty + 8 * buf);
+                            if (lane == 0) {
+                                if (kPair)
+                                    mbar_arrive_cluster(lead_tempty + 8 * buf);
+                                else
+                                    mbar_arrive(bar_tempty + 8 * buf);
+                            }
                         }
                     }
                     if (kWgrad) {
@@ -533,6 +695,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             }
             cp_async_wait<0>();
             if (!ok) break;
+            if (kPair && !x.valid) continue;   // the idle half of a pair: nothing to write
             const int64_t r = (int64_t)x.m0 + row;
             // ------------------------------------------- fused outputs ----
             if (kEpi == EPI_SILU) {
@@ -676,8 +839,24 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     }
     tc_fence_before();
     __syncthreads();
+    if (kPair) {
+        // After a timeout the peer may still have loads in flight that only the
+        // leader's barriers count: give them time to land before the pair
+        // leaves (loads finish in microseconds; this waits about a millisecond).
+        if (*abort_flag) {
+            const long long t0 = clock64();
+            while (clock64() - t0 < (1ll << 21)) {
+            }
+        }
+        cluster_sync_all();   // neither CTA frees its TMEM while the pair's MMAs may run
+    }
     tc_fence_after();
-    if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS));
+    if (warp == 1) {
+        if (kPair)
+            asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS));
+        else
+            asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS));
+    }
 }
 
 }  // namespace gemm
@@ -685,20 +864,50 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 // ------------------------------------------------------------------ host ----
 using namespace sm100;
 
-template <int kEpi, bool kGather = false>
+template <int kEpi, bool kGather = false, bool kPair = false>
 static int launch_one(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &c, const gemm::Args &args,
                       int grid, cudaStream_t s)
 {
+    auto kern = gemm::grouped_gemm_kernel<kEpi, kGather, kPair>;
+    constexpr int smem = gemm::smem_bytes<kEpi, kPair>();
     static bool configured = false;  // per process; attribute is per function
     if (!configured) {
-        if (cudaFuncSetAttribute(gemm::grouped_gemm_kernel<kEpi, kGather>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 gemm::smem_bytes<kEpi>()) != cudaSuccess)
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
             return MOE_ERR_CUDA;
         configured = true;
     }
-    gemm::grouped_gemm_kernel<kEpi, kGather><<<grid, gemm::NUM_THREADS, gemm::smem_bytes<kEpi>(), s>>>(a, b, c, args);
+    if (kPair) {   // clusters of two CTAs (one pair of SMs)
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(grid & ~1));
+        cfg.blockDim = dim3(gemm::NUM_THREADS);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, kern, a, b, c, args) != cudaSuccess) return MOE_ERR_CUDA;
+    } else {
+        kern<<<grid, gemm::NUM_THREADS, smem, s>>>(a, b, c, args);
+    }
     count_launch();
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// 1-SM (0), 2-SM (1) or chosen per call (-1) for the rows-mode GEMMs.
+static int g_variant = 0;
+void set_gemm_variant(int v) { g_variant = v; }
+
+// The 2-SM variant computes whole pairs of 128-row tiles; a segment with an
+// odd number of tiles leaves one half of its last pair idle.  It pays when
+// those idle halves (at most one per segment) are a small share of the rows.
+static bool use_pair(int n_seg, int64_t R_cap)
+{
+    if (g_variant >= 0) return g_variant == 1;
+    return (int64_t)n_seg * gemm::BM * 32 <= R_cap;
 }
 
 int launch_grouped_gemm(int op, const moe_dims &d, int64_t R_cap, const int32_t *offsets, int n_seg,
@@ -755,6 +964,17 @@ int launch_grouped_gemm(int op, const moe_dims &d, int64_t R_cap, const int32_t 
     if (op == MOE_GEMM_DOWN || op == MOE_GEMM_DGRAD_GATEUP) ok = make_store_map(&mC, g.out_bf16, a.N, R_cap, 2);
     if (!ok) return MOE_ERR_CUDA;
     const int grid = sm_count();
+    if (op != MOE_GEMM_WGRAD_DOWN && op != MOE_GEMM_WGRAD_GATEUP && use_pair(n_seg, R_cap)) {
+        // each CTA loads 128 rows of the 256-row B tile
+        const int64_t Kc = a.K, Nrows = (op == MOE_GEMM_GATEUP_SILU ? 2 * I : op == MOE_GEMM_DGRAD_DOWN_SILU ? I : D);
+        if (!make_map(&mB, g.b, Kc, E * Nrows, 128)) return MOE_ERR_CUDA;
+        switch (op) {
+        case MOE_GEMM_GATEUP_SILU: return launch_one<gemm::EPI_SILU, false, true>(mA, mB, mC, a, grid, s);
+        case MOE_GEMM_DOWN:
+        case MOE_GEMM_DGRAD_GATEUP: return launch_one<gemm::EPI_BF16, false, true>(mA, mB, mC, a, grid, s);
+        default: return launch_one<gemm::EPI_DSILU, false, true>(mA, mB, mC, a, grid, s);
+        }
+    }
     switch (op) {
     case MOE_GEMM_GATEUP_SILU: return launch_one<gemm::EPI_SILU>(mA, mB, mC, a, grid, s);
     case MOE_GEMM_DOWN:

@@ -10,6 +10,7 @@
 namespace moe {
 int launch_grouped_gemm(int op, const moe_dims &d, int64_t R_cap, const int32_t *offsets, int n_seg,
                         const moe_gemm_args &g, int *status, uint64_t budget, cudaStream_t s);
+void set_gemm_variant(int v);
 int launch_gateup_gather(const moe_dims &d, int64_t R_cap, const int32_t *offsets, const int32_t *src_idx,
                          const moe_gemm_args &g, int *status, uint64_t budget, cudaStream_t s);
 }
@@ -110,6 +111,13 @@ int moe_get_status(void *stream, int *out)
 void moe_set_wait_budget(uint64_t cycles) { g_wait_budget = cycles; }
 
 uint64_t moe_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int moe_set_gemm_variant(int variant)
+{
+    if (variant < -1 || variant > 1) return MOE_ERR_INVALID_ARG;
+    moe::set_gemm_variant(variant);
+    return MOE_OK;
+}
 
 int moe_route_topk(const float *logits, const moe_dims *d, int32_t *idx, float *w, void *stream)
 {
