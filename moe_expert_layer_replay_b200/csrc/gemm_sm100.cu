@@ -664,14 +664,19 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     if (kWgrad) {
                         // column scales of this chunk: 16-byte shared loads (a slot is
                         // 1536 B, the column part starts 512 B in)
+                        // (the scale products sa * sb[n] on two lanes at once: the
+                        // same fp32 products as two scalar multiplies)
                         const float4 *cs = reinterpret_cast<const float4 *>(d + BM + 128 * h + 32 * c);
 #pragma unroll
                         for (int i = 0; i < 32; i += 4) {
                             const float4 c4 = cs[i >> 2];
+                            float p0, p1, p2, p3;
+                            fmul2(p0, p1, sa, sa, c4.x, c4.y);
+                            fmul2(p2, p3, sa, sa, c4.z, c4.w);
                             ffma2(acc[32 * c + i], acc[32 * c + i + 1], __uint_as_float(cur[i]),
-                                  __uint_as_float(cur[i + 1]), sa * c4.x, sa * c4.y);
+                                  __uint_as_float(cur[i + 1]), p0, p1);
                             ffma2(acc[32 * c + i + 2], acc[32 * c + i + 3], __uint_as_float(cur[i + 2]),
-                                  __uint_as_float(cur[i + 3]), sa * c4.z, sa * c4.w);
+                                  __uint_as_float(cur[i + 3]), p2, p3);
                         }
                     } else {
                         const float sc = (kEpi == EPI_SILU && c >= 2) ? s1 : s0;
@@ -876,7 +881,7 @@ static int launch_one(const CUtensorMap &a, const CUtensorMap &b, const CUtensor
             return MOE_ERR_CUDA;
         configured = true;
     }
-    if (kPair) {   // clusters of two CTAs (one pair of SMs)
+    if (kPair) {   // clusters of two CTAs (one pair of SMs), as many as can be resident at once
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)(grid & ~1));
         cfg.blockDim = dim3(gemm::NUM_THREADS);
@@ -889,6 +894,15 @@ static int launch_one(const CUtensorMap &a, const CUtensorMap &b, const CUtensor
         attr[0].val.clusterDim.z = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
+        static int max_clusters = 0;   // per process: the device and the kernel's resources are fixed
+        if (max_clusters == 0) {
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, (void *)kern, &cfg) != cudaSuccess || n <= 0) return MOE_ERR_CUDA;
+            max_clusters = n;
+        }
+        // the tiles are dealt out statically by cluster index: every cluster
+        // must be resident at the same time
+        cfg.gridDim = dim3((unsigned)(2 * (grid / 2 < max_clusters ? grid / 2 : max_clusters)));
         if (cudaLaunchKernelEx(&cfg, kern, a, b, c, args) != cudaSuccess) return MOE_ERR_CUDA;
     } else {
         kern<<<grid, gemm::NUM_THREADS, smem, s>>>(a, b, c, args);

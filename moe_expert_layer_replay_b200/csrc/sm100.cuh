@@ -120,6 +120,15 @@ __device__ __forceinline__ void ffma2(float &a0, float &a1, float p0, float p1, 
         : "f"(p0), "f"(p1), "f"(s0), "f"(s1));
 }
 
+// (r0, r1) = (a0 * b0, a1 * b1) on two fp32 lanes at once (packed f32x2)
+__device__ __forceinline__ void fmul2(float &r0, float &r1, float a0, float a1, float b0, float b1)
+{
+    asm("{\n\t.reg .b64 a, b, r;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+        "mul.rn.f32x2 r, a, b;\n\tmov.b64 {%0, %1}, r;\n\t}"
+        : "=f"(r0), "=f"(r1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
 // TMA store of a 2D box from shared memory (bulk-group completion).
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t src, int32_t c0, int32_t c1)
 {
