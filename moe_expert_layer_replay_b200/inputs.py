@@ -19,10 +19,13 @@ W_gate -> W_up -> W_down -> dy):
     and the ``empty`` least popular experts at p = 0 (logit -inf), so the
     router itself samples the skewed, partly empty load;
   - ``replay_uniform``: inference logits U(0, 1) fp32; the payload is their
-    top-k order (this stands in for the inference-side capture, which this
-    library does not implement); the trainer's logits are the inference
-    logits plus 0.05 N(0, 1), so replay must override the trainer's own
-    choice.
+    top-k order; the trainer's logits are the inference logits plus
+    0.05 N(0, 1), so replay must override the trainer's own choice;
+  - ``replay_skew``: the same with inference logits log p_e + Gumbel,
+    p_e ~ (e+1)^-s (hot and cold experts).
+  The replay payloads are drawn here, as inputs, so that the kernels and the
+  oracle replay the same routing; the library's own router and capture
+  (moe_router_fwd, moe_capture_payload) are checked on their own.
 """
 from __future__ import annotations
 
@@ -66,6 +69,8 @@ WORKLOADS = {
                         routing="topk_zipf_skew", zipf=1.2, empty=4),
     "train": Workload("train", T=32768, D=7168, I=2048, E=32, k=8, routing="replay_uniform",
                       train=True),
+    "train_skew": Workload("train_skew", T=32768, D=7168, I=2048, E=32, k=8, routing="replay_skew",
+                           zipf=1.2, train=True),
 }
 
 
@@ -111,8 +116,12 @@ def _draw_routing(rng, wl: Workload, T: int) -> dict:
             g = rng.standard_exponential((T, k))
             w_in[layer] = (g / g.sum(axis=1, keepdims=True)).astype(np.float32)
         return {"payload": payload, "w_in": w_in}
-    if wl.routing == "replay_uniform":
-        z_inf = rng.random((T, E), dtype=np.float32)
+    if wl.routing in ("replay_uniform", "replay_skew"):
+        if wl.routing == "replay_uniform":
+            z_inf = rng.random((T, E), dtype=np.float32)
+        else:
+            p = (np.arange(1, E + 1, dtype=np.float64)) ** (-wl.zipf)
+            z_inf = (np.log(p / p.sum())[None, :] + _gumbel(rng, (T, E))).astype(np.float32)
         chosen = np.argsort(-z_inf, axis=1, kind="stable")[:, :k]
         payload = chosen.T[None].astype(np.int32).copy()
         z_train = (z_inf + np.float32(0.05) * rng.standard_normal((T, E), dtype=np.float32))
