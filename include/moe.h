@@ -216,6 +216,21 @@ int moe_quant_fp8_block(const uint16_t *in, int64_t rows, int64_t cols, int64_t 
                         int32_t blk_r, int32_t blk_c, uint8_t *q, float *s, uint8_t *qT,
                         float *sT, void *stream);
 
+/* NVFP4 block quantisation (the Blackwell 4-bit format named as future work
+ * in [P4 §Future work]) of in bf16 [rows][cols] (row stride ld elements,
+ * ld % 8 == 0, cols % 16 == 0, in 16-byte aligned, q 8-byte aligned):
+ *   amax (one float)  max |x| over the tensor;
+ *   s_g  (one float)  tensor scale fp32(2688 / amax) (1 if amax = 0);
+ *   sf [rows][cols/16] e4m3 block-scale codes: e4m3(RNE, satfinite)(
+ *                     fp32(fp32(amax_b / 6) * s_g)), amax_b over 16 elements;
+ *   q  [rows][cols/2] e2m1 codes, two per byte (element 2i in the low
+ *                     nibble): 0 where the block scale is 0, else e2m1(RNE,
+ *                     satfinite)(fp32(x * fp32(s_g / value(sf)))).
+ * Value of an element: e2m1(q) * value(sf) / s_g.  amax and s_g are device
+ * words the call writes (amax is zeroed first, then accumulated). */
+int moe_quant_nvfp4(const uint16_t *in, int64_t rows, int64_t cols, int64_t ld, uint8_t *q, uint8_t *sf,
+                    float *amax, float *s_g, void *stream);
+
 /* Expert weights (a5): 128x128 FP8 of W_gate, W_up [E][I][D] and W_down [E][D][I].
  *   wgu_q [E][2I][D], wgu_s [E][2I/128][D/128]: gate and up interleaved by
  *        128-row blocks (block 2b = gate rows 128b.., block 2b+1 = up rows 128b..);

@@ -22,7 +22,7 @@ EXPORTS = [
     "moe_quant_fp8_block", "moe_quant_weights", "moe_grouped_gemm_fp8", "moe_combine",
     "moe_combine_bwd", "moe_unpermute_reduce", "moe_permute_noalloc", "moe_kernel_launches",
     "moe_router_fwd", "moe_capture_payload", "moe_router_bwd_workspace_size", "moe_router_bwd",
-    "moe_grouped_gemm_fp8_seg", "moe_gateup_gather_fp8", "moe_set_gemm_variant",
+    "moe_grouped_gemm_fp8_seg", "moe_gateup_gather_fp8", "moe_set_gemm_variant", "moe_quant_nvfp4",
 ]
 
 
@@ -77,6 +77,7 @@ def lib() -> ctypes.CDLL:
             "moe_permute_noalloc": (ctypes.c_int, [P, D, P, P, P, P, P, P, P, P]),
             "moe_quant_fp8_block": (ctypes.c_int, [P, I64, I64, I64, I32, I32, P, P, P, P, P]),
             "moe_quant_weights": (ctypes.c_int, [P, P, P, D, P, P, P, P, P, P, P, P, P]),
+            "moe_quant_nvfp4": (ctypes.c_int, [P, I64, I64, I64, P, P, P, P, P]),
             "moe_grouped_gemm_fp8": (ctypes.c_int, [I32, D, P, ctypes.POINTER(GemmArgs), P]),
             "moe_grouped_gemm_fp8_seg": (ctypes.c_int, [I32, D, I64, P, I32, ctypes.POINTER(GemmArgs), P]),
             "moe_gateup_gather_fp8": (ctypes.c_int, [D, P, P, ctypes.POINTER(GemmArgs), P]),
@@ -192,6 +193,13 @@ def permute_noalloc(idx, d: Dims, counts, offsets, pos, src_idx, x, xq, xs, stre
 def quant_fp8_block(inp, rows, cols, ld, blk_r, blk_c, q, s, qT=None, sT=None, stream=None):
     _check("moe_quant_fp8_block", lib().moe_quant_fp8_block(_p(inp), int(rows), int(cols), int(ld), int(blk_r),
                                                             int(blk_c), _p(q), _p(s), _p(qT), _p(sT), _s(stream)))
+
+
+def quant_nvfp4(inp, rows, cols, ld, q, sf, amax, s_g, stream=None):
+    """NVFP4: packed e2m1 codes q [rows, cols/2], e4m3 block scales sf [rows, cols/16],
+    tensor amax and scale s_g (one float each, device)."""
+    _check("moe_quant_nvfp4", lib().moe_quant_nvfp4(_p(inp), int(rows), int(cols), int(ld), _p(q), _p(sf), _p(amax),
+                                                    _p(s_g), _s(stream)))
 
 
 def quant_weights(w_gate, w_up, w_down, d: Dims, wgu_q, wgu_s, wd_q, wd_s,

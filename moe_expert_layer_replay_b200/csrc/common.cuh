@@ -207,6 +207,8 @@ int launch_router_logits(const uint16_t *x, const uint16_t *w_r, int T, int D, i
 int launch_capture(const int32_t *idx, int T, int k, int layer, int32_t *payload, cudaStream_t s);
 int launch_router_bwd(const float *dz, const uint16_t *x, const uint16_t *w_r, int T, int D, int E,
                       const uint16_t *dx_in, uint16_t *dx, float *dw_r, void *ws, cudaStream_t s);
+int launch_quant_nvfp4(const uint16_t *in, int64_t rows, int64_t cols, int64_t ld, uint8_t *q, uint8_t *sf,
+                       float *amax, float *s_g, int sms, cudaStream_t s);
 int launch_combine(const uint16_t *Y, const float *w, const int32_t *pos, int T, int D, int k,
                    uint16_t *y, cudaStream_t s);
 int launch_combine_bwd(const uint16_t *dy, const uint16_t *Y, const float *w, const int32_t *pos,

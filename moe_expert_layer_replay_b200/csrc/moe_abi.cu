@@ -239,6 +239,17 @@ int moe_quant_fp8_block(const uint16_t *in, int64_t rows, int64_t cols, int64_t 
     return MOE_ERR_UNSUPPORTED;
 }
 
+int moe_quant_nvfp4(const uint16_t *in, int64_t rows, int64_t cols, int64_t ld, uint8_t *q, uint8_t *sf,
+                    float *amax, float *s_g, void *stream)
+{
+    if (rows < 0 || cols <= 0 || cols % 16 || ld < cols || ld % 8) return MOE_ERR_INVALID_ARG;
+    if (!amax || !s_g || !aligned4(amax) || !aligned4(s_g)) return MOE_ERR_INVALID_ARG;
+    if (rows > 0 && (!in || !q || !sf || !aligned16(in) || !aligned8(q))) return MOE_ERR_INVALID_ARG;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return moe::launch_quant_nvfp4(in, rows, cols, ld, q, sf, amax, s_g, sms, as_stream(stream));
+}
+
 int moe_quant_weights(const uint16_t *w_gate, const uint16_t *w_up, const uint16_t *w_down,
                       const moe_dims *d, uint8_t *wgu_q, float *wgu_s, uint8_t *wd_q, float *wd_s,
                       uint8_t *wguT_q, float *wguT_s, uint8_t *wdT_q, float *wdT_s, void *stream)
