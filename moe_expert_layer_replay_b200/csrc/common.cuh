@@ -147,6 +147,15 @@ __device__ __forceinline__ uint4 quant16(const float *v, float s)
     return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
+// Four codes (element i in byte i); a zero scale gives zero codes.
+__device__ __forceinline__ uint32_t quant4(const float *v, float s)
+{
+    if (s == 0.0f) return 0u;
+    float q[4];
+    quotients<4>(v, s, q);
+    return e4m3x2(q[0], q[1]) | (e4m3x2(q[2], q[3]) << 16);
+}
+
 __device__ __forceinline__ uint2 quant8(const float *v, float s)
 {
     if (s == 0.0f) return make_uint2(0, 0);

@@ -76,6 +76,11 @@ struct Lay {
     static constexpr int OFF_WS_BAR = OFF_WS + SC_SLOTS * WS_FLOATS * 4;  // sfull[SC_SLOTS], sempty[SC_SLOTS]
     static constexpr int OFF_TSTORE_SILU = OFF_EPI + 2 * 2 * 128 * 4;
     static constexpr int OFF_TSTORE_BF16 = OFF_EPI;
+    // pair mode, SILU: each epilogue thread's 64 h values (bf16) wait here for
+    // their quantisation, which runs during the next tile's K loop; rows of
+    // 128 h values padded to 272 bytes (16-byte accesses free of bank conflicts)
+    static constexpr int HSTAGE_ROW = 272;
+    static constexpr int OFF_HSTAGE = OFF_TSTORE_SILU + 8 * TSTORE_BUF;
 };
 
 enum Epi { EPI_SILU = 0, EPI_BF16 = 1, EPI_DSILU = 2, EPI_WGRAD = 3 };
@@ -84,7 +89,7 @@ template <int kEpi, bool kPair = false>
 constexpr int smem_bytes()
 {
     using L = Lay<kPair>;
-    return 1024 + (kEpi == EPI_SILU   ? L::OFF_TSTORE_SILU + 8 * TSTORE_BUF
+    return 1024 + (kEpi == EPI_SILU   ? L::OFF_TSTORE_SILU + 8 * TSTORE_BUF + (kPair ? 128 * L::HSTAGE_ROW : 0)
                    : kEpi == EPI_BF16 ? L::OFF_TSTORE_BF16 + 8 * 2 * TSTORE_BUF
                    : kEpi == EPI_WGRAD ? L::OFF_WS_BAR + 2 * SC_SLOTS * 8
                                        : L::OFF_EPI);  // + alignment slack
@@ -572,6 +577,35 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             ephase ^= 1;
             return r;
         };
+        // Pair mode, SILU: the h codes of the previous tile are made here, four
+        // per thread after each K block of the next tile (the h values wait in
+        // this thread's own slot of the staging area; the scale is known).
+        constexpr bool kDefer = kPair && kEpi == EPI_SILU;
+        int def_left = 0;           // h values of the deferred tile still to quantise
+        float def_s = 0.0f;
+        int def_m0 = 0, def_col = 0;
+        uint8_t *hst = smem + L::OFF_HSTAGE + row * L::HSTAGE_ROW + 128 * h;   // this thread's 64 h values
+        uint8_t *box = smem + OFF_TSTORE_SILU + ew * TSTORE_BUF;              // this warp's code box
+        auto defer_step = [&]() {
+            if (!kDefer || def_left == 0) return;   // warp-uniform
+            const int i0 = 64 - def_left;
+            if (i0 == 0) {
+                if (lane == 0) bulk_wait_read<0>();   // the box's previous store has read it
+                __syncwarp();
+            }
+            const uint2 hv = *reinterpret_cast<const uint2 *>(hst + 2 * i0);
+            const float v[4] = {bf16_lo(hv.x), bf16_hi(hv.x), bf16_lo(hv.y), bf16_hi(hv.y)};
+            *reinterpret_cast<uint32_t *>(box + lane * 64 + i0) = quant4(v, def_s);
+            def_left -= 4;
+            if (def_left == 0) {
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(&tmC, smem_u32(box), def_col, def_m0 + 32 * q);
+                    bulk_commit();
+                }
+            }
+        };
         for (int t = t_first; t < ntiles && ok; t += t_step, ++tcount) {
             const Tile x = tile_of<kWgrad, kPair>(t, p, offs_s, pps_s, rank);
             if (kWgrad && x.kb1 == x.kb0) continue;
@@ -695,6 +729,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                         wphase ^= 1;
                     }
                 }
+                defer_step();
                 buf ^= 1;
                 if (buf == 0) bphase ^= 1;
             }
@@ -729,18 +764,28 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 if (!epi_sync()) break;
                 amax = fmaxf(ax[row], ax[128 + row]);
                 const float s = block_scale(amax);
-                // this warp's 32 rows x 64 codes leave through one TMA store
-                uint8_t *sb = smem + OFF_TSTORE_SILU + ew * TSTORE_BUF;
-                if (lane == 0) bulk_wait_read<0>();  // the previous tile's store has read sb
-                __syncwarp();
+                if (kDefer) {
+                    while (def_left > 0) defer_step();   // a short tile: the previous codes first
 #pragma unroll
-                for (int i0 = 0; i0 < 64; i0 += 16)
-                    *reinterpret_cast<uint4 *>(sb + lane * 64 + i0) = quant16(&acc[i0], s);
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    tma_store_2d(&tmC, smem_u32(sb), (int32_t)icol, x.m0 + 32 * q);
-                    bulk_commit();
+                    for (int i0 = 0; i0 < 64; i0 += 8) *reinterpret_cast<uint4 *>(hst + 2 * i0) = pack8(&acc[i0]);
+                    def_left = 64;
+                    def_s = s;
+                    def_m0 = x.m0;
+                    def_col = (int)icol;
+                } else {
+                    // this warp's 32 rows x 64 codes leave through one TMA store
+                    uint8_t *sb = box;
+                    if (lane == 0) bulk_wait_read<0>();  // the previous tile's store has read sb
+                    __syncwarp();
+#pragma unroll
+                    for (int i0 = 0; i0 < 64; i0 += 16)
+                        *reinterpret_cast<uint4 *>(sb + lane * 64 + i0) = quant16(&acc[i0], s);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&tmC, smem_u32(sb), (int32_t)icol, x.m0 + 32 * q);
+                        bulk_commit();
+                    }
                 }
                 if (h == 0) p.out_s[(int64_t)x.nt * p.R_cap + r] = s;
                 if (p.out_bf16) {
@@ -839,6 +884,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 }
             }
         }
+        if (ok)
+            while (def_left > 0) defer_step();   // the last tile's codes
         cp_async_wait<0>();  // no copy into shared memory outlives the CTA
         if ((kEpi == EPI_SILU || kEpi == EPI_BF16) && lane == 0) bulk_wait_all();  // every TMA store has completed
     }
