@@ -277,7 +277,7 @@ def run_reference(args, wl_name):
     if rank != 0:
         return 0
     from moe_expert_layer_replay_b200.inputs import make_inputs
-    inp = make_inputs(wl_name, seed=args.seed)
+    inp = make_inputs(wl_name, seed=args.seed, T=args.tokens)
     wl = inp["workload"]
     tokens = args.ref_tokens or default_sample_tokens(wl, 4e10)
     wq = oracle_weights(inp)
@@ -360,7 +360,7 @@ def run_ours(args, wl_name):
         dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local))
     abi.lib()
 
-    inp = make_inputs(wl_name, seed=replica_seed(args.seed, rank))
+    inp = make_inputs(wl_name, seed=replica_seed(args.seed, rank), T=args.tokens)
     wl = inp["workload"]
     d = abi.dims(wl.T, wl.D, wl.I, wl.E, wl.k)
     W = layer.quantise_weights(d, _to_dev(inp["W_gate"]), _to_dev(inp["W_up"]), _to_dev(inp["W_down"]),
@@ -601,7 +601,7 @@ def run_kernels(args, names):
     fp8 = bf16_tf * FP8_OVER_BF16
     flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device="cuda")
     for name in names:
-        inp = make_inputs(name, seed=args.seed)
+        inp = make_inputs(name, seed=args.seed, T=args.tokens)
         wl = inp["workload"]
         T, D, I, E, k = wl.T, wl.D, wl.I, wl.E, wl.k
         R = T * k
@@ -731,6 +731,8 @@ def build_parser() -> argparse.ArgumentParser:
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="prefill")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override T (a smaller case of the same workload, e.g. for profiling)")
     ap.add_argument("--cpu-tokens", type=int, default=0, help="oracle sample size (0: sized to ~10 s)")
     ap.add_argument("--ref-tokens", type=int, default=0, help="oracle sample per reference step (0: ~1 s)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
