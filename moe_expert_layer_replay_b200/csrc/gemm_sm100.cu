@@ -60,9 +60,12 @@ constexpr int TSTORE_BUF = 32 * 64;
 //          epilogue warps), deeper than the operand ring
 //   DSILU  unused
 // Store buffers are read by TMA stores (32 rows x 64 bytes boxes, no swizzle).
-template <bool kPair>
+template <bool kPair, int kEpi = 0>
 struct Lay {
-    static constexpr int STAGES = kPair ? 5 : 4;
+    // the 2-SM bf16 output keeps four store boxes per warp (below) in place of
+    // the ring's fifth stage
+    static constexpr int STAGES = kPair ? (kEpi == 1 ? 4 : 5) : 4;
+    static constexpr int BF16_BUFS = kPair ? 4 : 2;   // store boxes per epilogue warp (bf16 output)
     static constexpr int B_BYTES = (kPair ? BN / 2 : BN) * BK;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int OFF_BAR = STAGES * STAGE_BYTES;
@@ -88,9 +91,9 @@ enum Epi { EPI_SILU = 0, EPI_BF16 = 1, EPI_DSILU = 2, EPI_WGRAD = 3 };
 template <int kEpi, bool kPair = false>
 constexpr int smem_bytes()
 {
-    using L = Lay<kPair>;
+    using L = Lay<kPair, kEpi>;
     return 1024 + (kEpi == EPI_SILU   ? L::OFF_TSTORE_SILU + 8 * TSTORE_BUF + (kPair ? 128 * L::HSTAGE_ROW : 0)
-                   : kEpi == EPI_BF16 ? L::OFF_TSTORE_BF16 + 8 * 2 * TSTORE_BUF
+                   : kEpi == EPI_BF16 ? L::OFF_TSTORE_BF16 + 8 * L::BF16_BUFS * TSTORE_BUF
                    : kEpi == EPI_WGRAD ? L::OFF_WS_BAR + 2 * SC_SLOTS * 8
                                        : L::OFF_EPI);  // + alignment slack
 }
@@ -99,6 +102,7 @@ static_assert(smem_bytes<EPI_SILU>() <= 232448 && smem_bytes<EPI_BF16>() <= 2324
                   smem_bytes<EPI_SILU, true>() <= 232448 && smem_bytes<EPI_BF16, true>() <= 232448 &&
                   smem_bytes<EPI_DSILU, true>() <= 232448,
               "shared memory budget");
+static_assert(EPI_BF16 == 1, "Lay's bf16 layout");
 static_assert(Lay<false>::OFF_EPI == 198656, "the one-SM layout is unchanged");
 
 struct Args {
@@ -300,7 +304,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 {
     constexpr bool kWgrad = (kEpi == EPI_WGRAD);
     static_assert(!(kPair && (kWgrad || kGather)), "the 2-SM variant covers the rows-mode GEMMs");
-    using L = Lay<kPair>;
+    using L = Lay<kPair, kEpi>;
     constexpr int STAGES = L::STAGES, STAGE_BYTES = L::STAGE_BYTES;
     constexpr int OFF_BAR = L::OFF_BAR, OFF_ABORT = L::OFF_ABORT, OFF_TMEM_SLOT = L::OFF_TMEM_SLOT;
     constexpr int OFF_OFFSETS = L::OFF_OFFSETS, OFF_AMAX = L::OFF_AMAX, OFF_WS = L::OFF_WS;
@@ -794,14 +798,20 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     for (int i0 = 0; i0 < 64; i0 += 8) *reinterpret_cast<uint4 *>(hb + i0) = pack8(&acc[i0]);
                 }
             } else if (kEpi == EPI_BF16) {
-                // 32-column chunks through two per-warp smem buffers, written to
-                // global memory by TMA stores that run while the warp moves on
+                // 32-column chunks through per-warp smem buffers (two, or one per
+                // chunk in the 2-SM layout), written to global memory by TMA
+                // stores that run while the warp moves on
+                constexpr int NB = L::BF16_BUFS;
                 const int64_t c0 = (int64_t)x.n0 + 128 * h;
                 if (c0 < p.N) {
 #pragma unroll
                     for (int ch = 0; ch < 4; ++ch) {
-                        uint8_t *buf = smem + OFF_TSTORE_BF16 + (ew * 2 + (ch & 1)) * TSTORE_BUF;
-                        if (lane == 0) bulk_wait_read<1>();  // the store that last read buf is done
+                        uint8_t *buf = smem + OFF_TSTORE_BF16 + (ew * NB + (ch % NB)) * TSTORE_BUF;
+                        if (NB == 2) {
+                            if (lane == 0) bulk_wait_read<1>();  // the store that last read buf is done
+                        } else if (ch == 0) {
+                            if (lane == 0) bulk_wait_read<0>();  // the previous tile's four stores have read theirs
+                        }
                         __syncwarp();
                         uint4 *w = reinterpret_cast<uint4 *>(buf + lane * 64);
 #pragma unroll
