@@ -344,6 +344,31 @@ class RoutingInput:
             self.t[k].copy_(other.t[k], non_blocking=True)
 
 
+def forward_calls(B, x, W, d, gather: bool, gemm1_events=None, stream=None):
+    """The layer's forward after routing, call by call (as layer.forward), with
+    the gate/up GEMM bracketed by CUDA events when a list is given."""
+    import torch
+
+    from moe_expert_layer_replay_b200 import abi
+    if gather:
+        abi.quant_fp8_block(x, d.T, d.D, d.D, 1, 128, B.xq_tok, B.xs_tok)
+        abi.permute(B.idx, d, B.counts, B.offsets, B.pos, B.src, None, None, None, None, None, B.ws)
+    else:
+        abi.permute(B.idx, d, B.counts, B.offsets, B.pos, B.src, x, B.xq, B.xs, None, None, B.ws)
+    if gemm1_events is not None:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+    if gather:
+        abi.gateup_gather_fp8(d, B.offsets, B.src, B.xq_tok, B.xs_tok, W.wgu_q, W.wgu_s, out_q=B.hq, out_s=B.hs)
+    else:
+        abi.grouped_gemm_fp8(abi.GEMM_GATEUP_SILU, d, B.offsets, B.xq, B.xs, W.wgu_q, W.wgu_s,
+                             out_q=B.hq, out_s=B.hs)
+    if gemm1_events is not None:
+        e1.record(stream)
+        gemm1_events.append((e0, e1))
+    abi.grouped_gemm_fp8(abi.GEMM_DOWN, d, B.offsets, B.hq, B.hs, W.wd_q, W.wd_s, out_bf16=B.Y)
+
+
 def run_ours(args, wl_name):
     import torch
     import torch.distributed as dist
@@ -365,7 +390,8 @@ def run_ours(args, wl_name):
     d = abi.dims(wl.T, wl.D, wl.I, wl.E, wl.k)
     W = layer.quantise_weights(d, _to_dev(inp["W_gate"]), _to_dev(inp["W_up"]), _to_dev(inp["W_down"]),
                                train=False)
-    B = layer.Buffers(d, "cuda", train=False)
+    gather = args.dispatch == "gather"
+    B = layer.Buffers(d, "cuda", train=False, gather=gather)
     x = _to_dev(inp["x"])
     rt = RoutingInput(inp)
     flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device="cuda")
@@ -376,16 +402,7 @@ def run_ours(args, wl_name):
     def step(timed_gemm: bool):
         for l in range(wl.L):
             rt.route(B, l)
-            abi.permute(B.idx, d, B.counts, B.offsets, B.pos, B.src, x, B.xq, B.xs, None, None, B.ws)
-            if timed_gemm:
-                e0, e1 = ev(), ev()
-                e0.record(stream)
-            abi.grouped_gemm_fp8(abi.GEMM_GATEUP_SILU, d, B.offsets, B.xq, B.xs, W.wgu_q, W.wgu_s,
-                                 out_q=B.hq, out_s=B.hs)
-            if timed_gemm:
-                e1.record(stream)
-                gemm1_events.append((e0, e1))
-            abi.grouped_gemm_fp8(abi.GEMM_DOWN, d, B.offsets, B.hq, B.hs, W.wd_q, W.wd_s, out_bf16=B.Y)
+            forward_calls(B, x, W, d, gather, gemm1_events if timed_gemm else None, stream)
             abi.combine(B.Y, B.w, B.pos, d, B.y)
 
     for _ in range(max(3, args.warmup)):
@@ -457,7 +474,7 @@ def run_ours(args, wl_name):
     # and every layer's output y back.  The copies run on two copy streams
     # ordered by events (double-buffered inputs; one y buffer per layer), so
     # they overlap the layer's kernels.
-    e2e_val, h2d, d2h = e2e_run(args, wl, d, W, inp, world, barrier)
+    e2e_val, h2d, d2h = e2e_run(args, wl, d, W, inp, world, barrier, gather)
 
     st = abi.get_status()
     if st != abi.OK:
@@ -480,6 +497,7 @@ def run_ours(args, wl_name):
             "config": {"workload": _workload_desc(wl), "tokens_per_step_per_gpu": wl.L * wl.T,
                        "launch": "CUDA graph of one step" if not args.no_graph else "eager",
                        "l2": "flushed between timed steps (512 MiB write, outside the timed events)",
+                       "dispatch": "gate/up GEMM gathers the token rows" if gather else "permuted FP8 copy",
                        "parallelism": "replicas" if world > 1 else "single GPU"},
             "roofline": {"bound": "tensor", "kernel": "grouped_gemm gate/up + SiLU + h-quant",
                          "achieved": achieved, "peak": fp8_peak, "unit": "TFLOP/s", "frac": achieved / fp8_peak,
@@ -511,14 +529,14 @@ def run_ours(args, wl_name):
     return 0
 
 
-def e2e_run(args, wl, d, W, inp, world, barrier):
+def e2e_run(args, wl, d, W, inp, world, barrier, gather=False):
     """Same metric through the public API with host buffers.  Returns
     (tokens/s over all ranks, H2D bytes per step, D2H bytes per step)."""
     import torch
 
     from moe_expert_layer_replay_b200 import abi, layer
 
-    B = layer.Buffers(d, "cuda", train=False)
+    B = layer.Buffers(d, "cuda", train=False, gather=gather)
     xh = torch.from_numpy(inp["x"].view(np.int16)).pin_memory()
     rth = RoutingInput(inp, dev=False)
     xd = [torch.empty(wl.T, wl.D, dtype=torch.int16, device="cuda") for _ in range(2)]
@@ -547,10 +565,7 @@ def e2e_run(args, wl, d, W, inp, world, barrier):
         x = xd[b].view(torch.bfloat16)
         for l in range(wl.L):
             rtd[b].route(B, l)
-            abi.permute(B.idx, d, B.counts, B.offsets, B.pos, B.src, x, B.xq, B.xs, None, None, B.ws)
-            abi.grouped_gemm_fp8(abi.GEMM_GATEUP_SILU, d, B.offsets, B.xq, B.xs, W.wgu_q, W.wgu_s,
-                                 out_q=B.hq, out_s=B.hs)
-            abi.grouped_gemm_fp8(abi.GEMM_DOWN, d, B.offsets, B.hq, B.hs, W.wd_q, W.wd_s, out_bf16=B.Y)
+            forward_calls(B, x, W, d, gather)
             abi.combine(B.Y, B.w, B.pos, d, yd[b][l])
             y_ready = Ev()
             y_ready.record(comp)
@@ -612,7 +627,7 @@ def run_kernels(args, names):
         train = wl.train
         wg, wu, wd = bfd(inp["W_gate"]), bfd(inp["W_up"]), bfd(inp["W_down"])
         W = layer.quantise_weights(d, wg, wu, wd, train=train)
-        B = layer.Buffers(d, "cuda", train=train)
+        B = layer.Buffers(d, "cuda", train=train, gather=True)
         x = bfd(inp["x"])
         if "payload" in inp:
             P = dev(inp["payload"])
@@ -642,6 +657,12 @@ def run_kernels(args, names):
             ("gemm down", lambda: abi.grouped_gemm_fp8(abi.GEMM_DOWN, d, B.offsets, B.hq, B.hs, W.wd_q, W.wd_s,
                                                        out_bf16=B.Y), "F", 2.0 * R * D * I),
             ("combine", lambda: abi.combine(B.Y, B.w, B.pos, d, B.y), "B", 2 * R * D + 8 * R + 2 * T * D),
+            # the gathered dispatch: x quantised once per token row, rows gathered by the GEMM
+            ("1x128 quant of the token rows", lambda: abi.quant_fp8_block(x, T, D, D, 1, 128, B.xq_tok, B.xs_tok),
+             "B", 2 * T * D + T * (D + D // 32)),
+            ("gemm gate/up gathering the token rows", lambda: abi.gateup_gather_fp8(
+                d, B.offsets, B.src, B.xq_tok, B.xs_tok, W.wgu_q, W.wgu_s, out_q=B.hq, out_s=B.hs), "F",
+             4.0 * R * D * I),
         ]
         if train:
             dy = bfd(inp["dy"])
@@ -737,6 +758,9 @@ def build_parser() -> argparse.ArgumentParser:
     ap.add_argument("--ref-tokens", type=int, default=0, help="oracle sample per reference step (0: ~1 s)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch the timed steps eagerly")
+    ap.add_argument("--dispatch", choices=["copy", "gather"], default="copy",
+                    help="copy: the permute writes the permuted FP8 rows; gather: the gate/up GEMM gathers "
+                         "them from the token rows")
     ap.add_argument("--gemm-variant", type=int, default=None,
                     help="grouped GEMM kernel: 0 one SM per tile, 1 the 2-SM MMA, -1 chosen per call "
                          "(default: the library's)")

@@ -172,8 +172,10 @@ int moe_route_replay(const int32_t *payload, int32_t L, int32_t layer, const moe
  *   src_idx [R_cap]   routed entry i = t*k+j held by each permuted row, -1 for
  *                     padding rows and rows >= offsets[E].
  * With x (bf16 [T][D]) non-NULL, also dispatches x in FP8:
- *   xq [R_cap][D] e4m3, xs [D/128][R_cap] fp32: 1x128 blocks of row pos[t][j]
- *   are those of x[t]; padding rows get codes 0 and scale 0.
+ *   xq [R_cap][D] e4m3, xs [D/128][R_cap] fp32 (both or neither): 1x128
+ *   blocks of row pos[t][j] are those of x[t]; padding rows get codes 0 and
+ *   scale 0 (NULL when the gate/up GEMM gathers the token rows itself,
+ *   moe_gateup_gather_fp8);
  *   xqT [D][R_cap], xsT [R_cap/128][D] (both nullable, align must be 128;
  *   with T > 0 they need x): 128x1 blocks of the permuted rows, for the
  *   weight gradient.  With T = 0 there is no row to dispatch and x may be

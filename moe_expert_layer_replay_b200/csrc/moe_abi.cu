@@ -198,7 +198,8 @@ int moe_permute(const int32_t *idx, const moe_dims *d, int32_t *counts, int32_t 
     if (!counts || !offsets || !src_idx || !ws) return MOE_ERR_INVALID_ARG;
     if (d->T > 0 && (!idx || !pos)) return MOE_ERR_INVALID_ARG;
     if (ws_bytes < moe_permute_workspace_size(d) || !aligned16(ws)) return MOE_ERR_INVALID_ARG;
-    if (x && (!xq || !xs || !aligned16(x) || !aligned16(xq) || !aligned4(xs))) return MOE_ERR_INVALID_ARG;
+    if ((xq == nullptr) != (xs == nullptr) || (xq && !x)) return MOE_ERR_INVALID_ARG;
+    if (x && (!aligned16(x) || (xq && (!aligned16(xq) || !aligned4(xs))))) return MOE_ERR_INVALID_ARG;
     if ((xqT == nullptr) != (xsT == nullptr)) return MOE_ERR_INVALID_ARG;
     if (xqT && ((d->T > 0 && !x) || d->align != 128 || !aligned16(xqT))) return MOE_ERR_INVALID_ARG;
     int *sp = status_ptr();
@@ -208,7 +209,7 @@ int moe_permute(const int32_t *idx, const moe_dims *d, int32_t *counts, int32_t 
     st = moe::launch_permute_index(idx, d->T, d->k, d->E, d->align, counts, offsets, pos, src_idx,
                                    R_cap, ws, sp, s);
     if (st || !x) return st;
-    st = moe::launch_dispatch_quant(x, d->T, d->D, pos, d->k, xq, xs, R_cap, counts, offsets, d->E, s);
+    if (xq) st = moe::launch_dispatch_quant(x, d->T, d->D, pos, d->k, xq, xs, R_cap, counts, offsets, d->E, s);
     if (st || !xqT) return st;
     return moe::launch_quant_rows128(x, d->D, src_idx, d->k, R_cap, d->D, R_cap, xqT, xsT, s);
 }

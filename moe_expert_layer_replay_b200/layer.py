@@ -52,9 +52,10 @@ class Buffers:
     """Every device buffer one layer pass needs, sized from the dims alone
     (R_cap rows bound the permuted rows, so nothing is read back)."""
 
-    def __init__(self, d: abi.Dims, device, train: bool):
+    def __init__(self, d: abi.Dims, device, train: bool, gather: bool = False):
         self.d = d
         self.train = train
+        self.gather = gather
         T, D, I, E, k = d.T, d.D, d.I, d.E, d.k
         R = abi.rows_capacity(d)
         self.R_cap = R
@@ -72,6 +73,9 @@ class Buffers:
         self.hs = torch.empty(I // 128, R, dtype=F32, **z)
         self.Y = torch.empty(R, D, dtype=BF16, **z)
         self.y = torch.empty(T, D, dtype=BF16, **z)
+        if gather:   # 1x128 FP8 of the token rows, read by the gathering gate/up GEMM
+            self.xq_tok = torch.empty(T, D, dtype=U8, **z)
+            self.xs_tok = torch.empty(D // 128, T, dtype=F32, **z)
         if train:
             self.gu = torch.empty(R, 2 * I, dtype=BF16, **z)
             self.h = torch.empty(R, I, dtype=BF16, **z)
@@ -107,14 +111,24 @@ def route(B: Buffers, logits=None, payload=None, layer: int = 0, w_in=None, stre
 
 def forward(B: Buffers, x, W: Weights, stream=None, h_out=None):
     """a3-a8 after routing.  Returns B.y.  ``h_out`` (optional, [R_cap, I]
-    bf16) receives h; training runs keep h in B.h."""
+    bf16) receives h; training runs keep h in B.h.  Buffers made with
+    gather=True quantise the token rows once and let the gate/up GEMM gather
+    its rows (no permuted FP8 copy; the forward's results are the same)."""
     d = B.d
     t = B.train
-    abi.permute(B.idx, d, B.counts, B.offsets, B.pos, B.src, x, B.xq, B.xs,
-                B.xqT if t else None, B.xsT if t else None, B.ws, stream=stream)
-    abi.grouped_gemm_fp8(abi.GEMM_GATEUP_SILU, d, B.offsets, B.xq, B.xs, W.wgu_q, W.wgu_s,
-                         aux=B.gu if t else None, out_q=B.hq, out_s=B.hs,
-                         out_bf16=B.h if t else h_out, stream=stream)
+    if B.gather:
+        abi.quant_fp8_block(x, d.T, d.D, d.D, 1, 128, B.xq_tok, B.xs_tok, stream=stream)
+        abi.permute(B.idx, d, B.counts, B.offsets, B.pos, B.src, x if t else None, None, None,
+                    B.xqT if t else None, B.xsT if t else None, B.ws, stream=stream)
+        abi.gateup_gather_fp8(d, B.offsets, B.src, B.xq_tok, B.xs_tok, W.wgu_q, W.wgu_s,
+                              aux=B.gu if t else None, out_q=B.hq, out_s=B.hs,
+                              out_bf16=B.h if t else h_out, stream=stream)
+    else:
+        abi.permute(B.idx, d, B.counts, B.offsets, B.pos, B.src, x, B.xq, B.xs,
+                    B.xqT if t else None, B.xsT if t else None, B.ws, stream=stream)
+        abi.grouped_gemm_fp8(abi.GEMM_GATEUP_SILU, d, B.offsets, B.xq, B.xs, W.wgu_q, W.wgu_s,
+                             aux=B.gu if t else None, out_q=B.hq, out_s=B.hs,
+                             out_bf16=B.h if t else h_out, stream=stream)
     abi.grouped_gemm_fp8(abi.GEMM_DOWN, d, B.offsets, B.hq, B.hs, W.wd_q, W.wd_s, out_bf16=B.Y, stream=stream)
     abi.combine(B.Y, B.w, B.pos, d, B.y, stream=stream)
     return B.y

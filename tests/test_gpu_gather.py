@@ -80,3 +80,28 @@ def test_gateup_gather_equals_dispatched(A, orc, case):
     idx, w = orc.route_topk(z, k)
     fw = OL.forward(x, idx, w, Wg, Wu, Wd)
     close(bf(host(h2)[:Rp]), bf(fw["h"]), bf16=True, what="h (gathered) vs oracle")
+
+
+def test_layer_forward_backward_gathered_equals_copy(A):
+    """The whole layer, forward and backward, with Buffers(gather=True): the
+    same outputs and gradients, bit for bit, as the permuted-copy path."""
+    from moe_expert_layer_replay_b200 import layer
+    rng = np.random.default_rng(320)
+    T, D, I, E, k = 700, 512, 256, 8, 3
+    z = rng.standard_normal((T, E)).astype(np.float32)
+    x = rand_bf16(rng, (T, D))
+    Wg, Wu, Wd = rand_bf16(rng, (E, I, D), 0.02), rand_bf16(rng, (E, I, D), 0.02), rand_bf16(rng, (E, D, I), 0.02)
+    dy = rand_bf16(rng, (T, D), 0.01)
+    d = A.dims(T, D, I, E, k)
+    outs = []
+    for gather in (False, True):
+        W = layer.quantise_weights(d, dev(Wg), dev(Wu), dev(Wd), train=True)
+        B = layer.Buffers(d, "cuda", train=True, gather=gather)
+        layer.route(B, logits=dev(z))
+        layer.forward(B, dev(x), W)
+        layer.backward(B, dev(dy), W, router_logits=True)
+        torch.cuda.synchronize()
+        assert A.get_status() == A.OK
+        outs.append({n: host(getattr(B, n)) for n in ("y", "hq", "h", "dx", "d_w", "d_logits", "dWd", "dWgu")})
+    for n in outs[0]:
+        same_bits(outs[1][n], outs[0][n], f"{n} (gathered vs copy)")
