@@ -734,6 +734,7 @@ def run_kernels(args, names):
             raise RuntimeError("device status after the timed replays")
         gf = [o for o in out if "flop" in o]
         line = {"kernels_report": _workload_desc(wl), "R": R, "R_pad": R_pad,
+                "gemm_pair_clusters": abi.gemm_pair_clusters(),
                 "peaks": {"hbm_gbs": hbm, "fp8_tflops": fp8, "source": src},
                 "gemm_tflops": round(sum(o["flop"] for o in gf) / (sum(o["us"] for o in gf) * 1e-6) / 1e12, 1),
                 "stages": out}

@@ -99,6 +99,11 @@ uint64_t moe_kernel_launches(void);
  * MOE_ERR_INVALID_ARG for any other value. */
 int moe_set_gemm_variant(int variant);
 
+/* Clusters (CTA pairs) of the last 2-SM GEMM launch: the pairs the device can
+ * hold at once, at most half the SMs (0 before any 2-SM launch).  For
+ * accounting only. */
+int moe_gemm_pair_clusters(void);
+
 /* ------------------------------------------------------------------------ */
 /* a1  Top-k routing  [P1 §Drift og omkostninger i realiteten]               */
 /* ------------------------------------------------------------------------ */

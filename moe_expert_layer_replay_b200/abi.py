@@ -23,6 +23,7 @@ EXPORTS = [
     "moe_combine_bwd", "moe_unpermute_reduce", "moe_permute_noalloc", "moe_kernel_launches",
     "moe_router_fwd", "moe_capture_payload", "moe_router_bwd_workspace_size", "moe_router_bwd",
     "moe_grouped_gemm_fp8_seg", "moe_gateup_gather_fp8", "moe_set_gemm_variant", "moe_quant_nvfp4",
+    "moe_gemm_pair_clusters",
 ]
 
 
@@ -67,6 +68,7 @@ def lib() -> ctypes.CDLL:
             "moe_set_wait_budget": (None, [U64]),
             "moe_kernel_launches": (U64, []),
             "moe_set_gemm_variant": (ctypes.c_int, [ctypes.c_int]),
+            "moe_gemm_pair_clusters": (ctypes.c_int, []),
             "moe_route_topk": (ctypes.c_int, [P, D, P, P, P]),
             "moe_route_replay": (ctypes.c_int, [P, I32, I32, D, P, P, P, P, P]),
             "moe_router_fwd": (ctypes.c_int, [P, P, D, P, P, P, P]),
@@ -142,6 +144,11 @@ def set_wait_budget(cycles: int) -> None:
 def set_gemm_variant(variant: int) -> None:
     """0: one-SM tiles (default), 1: the 2-SM MMA, -1: chosen per call."""
     _check("moe_set_gemm_variant", lib().moe_set_gemm_variant(int(variant)))
+
+
+def gemm_pair_clusters() -> int:
+    """CTA pairs of the last 2-SM GEMM launch (0 before any)."""
+    return int(lib().moe_gemm_pair_clusters())
 
 
 def kernel_launches() -> int:

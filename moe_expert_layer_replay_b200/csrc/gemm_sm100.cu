@@ -193,10 +193,13 @@ __device__ __forceinline__ void cluster_sync_all()
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-// arrive on an mbarrier given by its shared::cluster address (any CTA of the cluster)
+// arrive on an mbarrier given by its shared::cluster address (any CTA of the
+// cluster).  The arriving thread's TMEM reads have completed (tcgen05.wait::ld)
+// and are fenced (tcgen05.fence::before_thread_sync); nothing else needs to be
+// made visible to the peer, so the arrive keeps the default CTA-scope order.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar)
 {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
 // TMA tile load into this CTA's shared memory whose completion is counted on
@@ -926,6 +929,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 // ------------------------------------------------------------------ host ----
 using namespace sm100;
 
+// 1-SM (0), 2-SM (1) or chosen per call (-1) for the rows-mode GEMMs.
+static int g_variant = 0;
+void set_gemm_variant(int v) { g_variant = v; }
+static int g_pair_clusters = 0;   // clusters of the last 2-SM launch
+int pair_clusters() { return g_pair_clusters; }
+
 template <int kEpi, bool kGather = false, bool kPair = false>
 static int launch_one(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &c, const gemm::Args &args,
                       int grid, cudaStream_t s)
@@ -960,6 +969,7 @@ static int launch_one(const CUtensorMap &a, const CUtensorMap &b, const CUtensor
         // the tiles are dealt out statically by cluster index: every cluster
         // must be resident at the same time
         cfg.gridDim = dim3((unsigned)(2 * (grid / 2 < max_clusters ? grid / 2 : max_clusters)));
+        g_pair_clusters = (int)(cfg.gridDim.x / 2);
         if (cudaLaunchKernelEx(&cfg, kern, a, b, c, args) != cudaSuccess) return MOE_ERR_CUDA;
     } else {
         kern<<<grid, gemm::NUM_THREADS, smem, s>>>(a, b, c, args);
@@ -968,9 +978,6 @@ static int launch_one(const CUtensorMap &a, const CUtensorMap &b, const CUtensor
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
-// 1-SM (0), 2-SM (1) or chosen per call (-1) for the rows-mode GEMMs.
-static int g_variant = 0;
-void set_gemm_variant(int v) { g_variant = v; }
 
 // The 2-SM variant computes whole pairs of 128-row tiles; a segment with an
 // odd number of tiles leaves one half of its last pair idle.  It pays when

@@ -11,6 +11,7 @@ namespace moe {
 int launch_grouped_gemm(int op, const moe_dims &d, int64_t R_cap, const int32_t *offsets, int n_seg,
                         const moe_gemm_args &g, int *status, uint64_t budget, cudaStream_t s);
 void set_gemm_variant(int v);
+int pair_clusters();
 int launch_gateup_gather(const moe_dims &d, int64_t R_cap, const int32_t *offsets, const int32_t *src_idx,
                          const moe_gemm_args &g, int *status, uint64_t budget, cudaStream_t s);
 }
@@ -118,6 +119,8 @@ int moe_set_gemm_variant(int variant)
     moe::set_gemm_variant(variant);
     return MOE_OK;
 }
+
+int moe_gemm_pair_clusters(void) { return moe::pair_clusters(); }
 
 int moe_route_topk(const float *logits, const moe_dims *d, int32_t *idx, float *w, void *stream)
 {
