@@ -73,7 +73,8 @@ struct Lay {
     static constexpr int OFF_ABORT = OFF_TMEM_SLOT + 4;
     static constexpr int OFF_OFFSETS = OFF_BAR + 256;
     static constexpr int OFF_PAIRS = OFF_OFFSETS + 1040;
-    static constexpr int OFF_EPI = (OFF_PAIRS + (kPair ? 1040 : 0) + 1023) / 1024 * 1024;
+    static constexpr int OFF_DEFXY = OFF_PAIRS + (kPair ? 1040 : 0);   // SILU: [8 warps][2] ints
+    static constexpr int OFF_EPI = (OFF_DEFXY + 64 + 1023) / 1024 * 1024;
     static constexpr int OFF_AMAX = OFF_EPI;
     static constexpr int OFF_WS = OFF_EPI;
     static constexpr int OFF_WS_BAR = OFF_WS + SC_SLOTS * WS_FLOATS * 4;  // sfull[SC_SLOTS], sempty[SC_SLOTS]
@@ -103,6 +104,8 @@ static_assert(smem_bytes<EPI_SILU>() <= 232448 && smem_bytes<EPI_BF16>() <= 2324
                   smem_bytes<EPI_DSILU, true>() <= 232448,
               "shared memory budget");
 static_assert(EPI_BF16 == 1, "Lay's bf16 layout");
+static_assert(Lay<false>::OFF_DEFXY + 64 <= Lay<false>::OFF_EPI && Lay<true>::OFF_DEFXY + 64 <= Lay<true>::OFF_EPI,
+              "deferred-store coordinates below the epilogue region");
 static_assert(Lay<false>::OFF_EPI == 198656, "the one-SM layout is unchanged");
 
 struct Args {
@@ -584,14 +587,22 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             ephase ^= 1;
             return r;
         };
-        // Pair mode, SILU: the h codes of the previous tile are made here, four
-        // per thread after each K block of the next tile (the h values wait in
-        // this thread's own slot of the staging area; the scale is known).
-        constexpr bool kDefer = kPair && kEpi == EPI_SILU;
+        // SILU: the h codes of a tile are made during the next tile's K loop,
+        // four per thread after each K block (the scale is known by then).  The
+        // h values wait in this thread's own slot of a shared-memory staging
+        // area (2-SM layout) or in the bf16 h output the caller asked for
+        // (one-SM layout; read back one step ahead, from L2); without either
+        // the codes are made at once.
+        constexpr bool kDefer = kEpi == EPI_SILU;
+        const bool defer_on = kDefer && (kPair || p.out_bf16 != nullptr);
         int def_left = 0;           // h values of the deferred tile still to quantise
         float def_s = 0.0f;
-        int def_m0 = 0, def_col = 0;
-        uint8_t *hst = smem + L::OFF_HSTAGE + row * L::HSTAGE_ROW + 128 * h;   // this thread's 64 h values
+        // the deferred tile's store coordinates (column, first row), per warp, kept in
+        // shared memory: the K loop's registers are all taken
+        int *def_xy = reinterpret_cast<int *>(smem + L::OFF_DEFXY) + 2 * ew;
+        const uint8_t *def_src = nullptr;   // this thread's 64 h values (bf16) of the deferred tile
+        uint2 def_next = make_uint2(0, 0);  // the next four, loaded one step ahead
+        uint8_t *hst = smem + L::OFF_HSTAGE + row * L::HSTAGE_ROW + 128 * h;   // 2-SM staging slot
         uint8_t *box = smem + OFF_TSTORE_SILU + ew * TSTORE_BUF;              // this warp's code box
         auto defer_step = [&]() {
             if (!kDefer || def_left == 0) return;   // warp-uniform
@@ -600,7 +611,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 if (lane == 0) bulk_wait_read<0>();   // the box's previous store has read it
                 __syncwarp();
             }
-            const uint2 hv = *reinterpret_cast<const uint2 *>(hst + 2 * i0);
+            const uint2 hv = def_next;
+            if (i0 + 4 < 64) def_next = *reinterpret_cast<const uint2 *>(def_src + 2 * (i0 + 4));
             const float v[4] = {bf16_lo(hv.x), bf16_hi(hv.x), bf16_lo(hv.y), bf16_hi(hv.y)};
             *reinterpret_cast<uint32_t *>(box + lane * 64 + i0) = quant4(v, def_s);
             def_left -= 4;
@@ -608,7 +620,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    tma_store_2d(&tmC, smem_u32(box), def_col, def_m0 + 32 * q);
+                    tma_store_2d(&tmC, smem_u32(box), def_xy[0], def_xy[1] + 32 * q);
                     bulk_commit();
                 }
             }
@@ -771,14 +783,21 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 if (!epi_sync()) break;
                 amax = fmaxf(ax[row], ax[128 + row]);
                 const float s = block_scale(amax);
-                if (kDefer) {
+                if (defer_on) {
                     while (def_left > 0) defer_step();   // a short tile: the previous codes first
+                    // the h row: to the staging slot, or to the caller's h output (written
+                    // now rather than below), then read back by the deferred steps
+                    uint8_t *dst = kPair ? hst : reinterpret_cast<uint8_t *>(p.out_bf16 + r * I + icol);
 #pragma unroll
-                    for (int i0 = 0; i0 < 64; i0 += 8) *reinterpret_cast<uint4 *>(hst + 2 * i0) = pack8(&acc[i0]);
+                    for (int i0 = 0; i0 < 64; i0 += 8) *reinterpret_cast<uint4 *>(dst + 2 * i0) = pack8(&acc[i0]);
+                    def_src = dst;
+                    def_next = *reinterpret_cast<const uint2 *>(dst);
                     def_left = 64;
                     def_s = s;
-                    def_m0 = x.m0;
-                    def_col = (int)icol;
+                    if (lane == 0) {
+                        def_xy[0] = (int)icol;
+                        def_xy[1] = x.m0;
+                    }
                 } else {
                     // this warp's 32 rows x 64 codes leave through one TMA store
                     uint8_t *sb = box;
@@ -795,7 +814,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     }
                 }
                 if (h == 0) p.out_s[(int64_t)x.nt * p.R_cap + r] = s;
-                if (p.out_bf16) {
+                if (p.out_bf16 && !(defer_on && !kPair)) {   // (the one-SM deferral wrote it already)
                     uint16_t *hb = p.out_bf16 + r * I + icol;
 #pragma unroll
                     for (int i0 = 0; i0 < 64; i0 += 8) *reinterpret_cast<uint4 *>(hb + i0) = pack8(&acc[i0]);
