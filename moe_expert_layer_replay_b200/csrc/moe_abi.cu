@@ -201,7 +201,7 @@ int moe_permute(const int32_t *idx, const moe_dims *d, int32_t *counts, int32_t 
     if (!counts || !offsets || !src_idx || !ws) return MOE_ERR_INVALID_ARG;
     if (d->T > 0 && (!idx || !pos)) return MOE_ERR_INVALID_ARG;
     if (ws_bytes < moe_permute_workspace_size(d) || !aligned16(ws)) return MOE_ERR_INVALID_ARG;
-    if ((xq == nullptr) != (xs == nullptr) || (xq && !x)) return MOE_ERR_INVALID_ARG;
+    if ((xq == nullptr) != (xs == nullptr) || (xq && !x && d->T > 0)) return MOE_ERR_INVALID_ARG;
     if (x && (!aligned16(x) || (xq && (!aligned16(xq) || !aligned4(xs))))) return MOE_ERR_INVALID_ARG;
     if ((xqT == nullptr) != (xsT == nullptr)) return MOE_ERR_INVALID_ARG;
     if (xqT && ((d->T > 0 && !x) || d->align != 128 || !aligned16(xqT))) return MOE_ERR_INVALID_ARG;
