@@ -616,7 +616,7 @@ def run_kernels(args, names):
     fp8 = bf16_tf * FP8_OVER_BF16
     flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device="cuda")
     for name in names:
-        inp = make_inputs(name, seed=args.seed, T=args.tokens)
+        inp = make_inputs(name, seed=args.seed, T=args.tokens, E=args.experts)
         wl = inp["workload"]
         T, D, I, E, k = wl.T, wl.D, wl.I, wl.E, wl.k
         R = T * k
@@ -698,6 +698,11 @@ def run_kernels(args, names):
         torch.cuda.synchronize()
         if abi.get_status() != abi.OK:
             raise RuntimeError("device status after the warm-up pass")
+        if args.once:   # one eager launch of every stage (for a profiler), no timing
+            print(json.dumps({"kernels_once": _workload_desc(wl), "stages": [n for n, _, _, _ in st]}), flush=True)
+            del B, W, x
+            torch.cuda.empty_cache()
+            continue
         gs = torch.cuda.Stream()
         out = []
         for sname, f, kind, units in st:
@@ -755,6 +760,8 @@ def build_parser() -> argparse.ArgumentParser:
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--tokens", type=int, default=None,
                     help="override T (a smaller case of the same workload, e.g. for profiling)")
+    ap.add_argument("--experts", type=int, default=None,
+                    help="with --kernels: override E (a smaller case of the same workload, e.g. for profiling)")
     ap.add_argument("--cpu-tokens", type=int, default=0, help="oracle sample size (0: sized to ~10 s)")
     ap.add_argument("--ref-tokens", type=int, default=0, help="oracle sample per reference step (0: ~1 s)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -763,8 +770,11 @@ def build_parser() -> argparse.ArgumentParser:
                     help="copy: the permute writes the permuted FP8 rows; gather: the gate/up GEMM gathers "
                          "them from the token rows")
     ap.add_argument("--gemm-variant", type=int, default=None,
-                    help="grouped GEMM kernel: 0 one SM per tile, 1 the 2-SM MMA, -1 chosen per call "
+                    help="grouped GEMM kernel: 0 one SM per tile, 1 the 2-SM MMA, 2 the 2-SM MMA reading "
+                         "TMEM one chunk ahead, 3 one SM reading one chunk ahead, -1 chosen per call "
                          "(default: the library's)")
+    ap.add_argument("--once", action="store_true",
+                    help="with --kernels: run every stage once, eagerly and untimed (for a profiler)")
     ap.add_argument("--kernels", default=None,
                     help="comma-separated workloads: per-stage device times and roofline fractions instead "
                          "of the bench line")

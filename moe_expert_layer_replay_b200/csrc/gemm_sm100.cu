@@ -18,6 +18,15 @@
 //              scale; per-column for wgrad) and add into fp32 registers; the
 //              freed TMEM buffer is handed back while the MMA fills the
 //              other.  After the last K block: the fused output step.
+// 2-SM variant (rows mode): clusters of two CTAs on two SMs; the leader issues
+// tcgen05.mma.cta_group::2 with M = 256 (each CTA's own 128 rows of A) and
+// N = 128, each K block as two column halves into separate 128-column TMEM
+// slots (four slots in all).  The epilogue warpgroup of one half releases its
+// slot while the other half's MMAs still run, so the MMA-to-release round trip
+// has three half-K-blocks of MMA work to hide behind instead of one K block.
+// Each CTA loads its own operand rows (no multicast); per SM and K block the
+// shared memory moves 32 KB of TMA writes and 48 KB of MMA reads instead of
+// 48 + 48 KB in the one-SM tile.
 // The scales are arbitrary fp32 (amax/448), so they cannot ride in the
 // hardware block-scaled MMA (which takes power-of-two UE8M0 scales); each
 // K block's partial product is promoted in fp32 instead.
@@ -151,10 +160,13 @@ __device__ __forceinline__ void mma_f8(uint32_t tmem_d, uint64_t a, uint64_t b, 
 }
 
 // The 2-SM MMA (cta_group::2): M = 256 over the CTA pair (128 rows of A in
-// each CTA's shared memory at the same offset), N = 256 (each CTA holds 128
-// rows of B: the leader rows 0-127, the peer rows 128-255), D in each CTA's
-// TMEM (its own 128 rows).  Issued by the leader CTA only.
-constexpr uint32_t IDESC_PAIR = (1u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(BN >> 3) << 17) |
+// each CTA's shared memory at the same offset), N = 128: each CTA supplies 64
+// rows of B from the same offset, the leader's give D columns 0-63 and the
+// peer's columns 64-127; D lands in each CTA's TMEM (its own 128 rows).
+// Issued by the leader CTA only, twice per K block (the two column halves of
+// the 256-column tile, each into its own TMEM slot).
+constexpr int BN_HALF = BN / 2;
+constexpr uint32_t IDESC_PAIR = (1u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(BN_HALF >> 3) << 17) |
                                 ((uint32_t)(2 * BM >> 4) << 24);
 
 __device__ __forceinline__ void mma_f8_pair(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t accum)
@@ -303,7 +315,7 @@ __device__ __forceinline__ Tile tile_of(int t, const Args &p, const int *offs_s,
 }
 
 // --------------------------------------------------------------- kernel ----
-template <int kEpi, bool kGather = false, bool kPair = false>
+template <int kEpi, bool kGather = false, bool kPair = false, bool kAhead = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmC, const Args p)
@@ -321,9 +333,13 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     const uint32_t sbase = smem_u32(smem);
     const uint32_t bar_full = sbase + OFF_BAR;           // [STAGES]
     const uint32_t bar_empty = bar_full + STAGES * 8;     // [STAGES]
-    const uint32_t bar_tfull = bar_empty + STAGES * 8;    // [2]
-    const uint32_t bar_tempty = bar_tfull + 2 * 8;        // [2]
-    const uint32_t bar_drain = bar_tempty + 2 * 8;
+    // TMEM slots: two 256-column buffers; in pair mode each buffer is two
+    // 128-column slots (one per MMA column half), slot 2 * buffer + half
+    constexpr int NQ = kPair ? 4 : 2;
+    static_assert(2 * STAGES * 8 + 2 * NQ * 8 + 16 <= OFF_TMEM_SLOT - OFF_BAR, "barrier area");
+    const uint32_t bar_tfull = bar_empty + STAGES * 8;    // [NQ]
+    const uint32_t bar_tempty = bar_tfull + NQ * 8;       // [NQ]
+    const uint32_t bar_drain = bar_tempty + NQ * 8;
     const uint32_t bar_epi = bar_drain + 8;  // the 256 epilogue threads meet here
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_ABORT);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_TMEM_SLOT);
@@ -364,9 +380,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 mbar_init(bar_sfull + 8 * s, 1);
                 mbar_init(bar_sempty + 8 * s, EPI_THREADS / 32);
             }
-        for (int b = 0; b < 2; ++b) {
+        // a slot is released by the epilogue warps that read it: all eight
+        // (one SM), or one warpgroup in each CTA of the pair (2 x 4)
+        for (int b = 0; b < NQ; ++b) {
             mbar_init(bar_tfull + 8 * b, 1);
-            mbar_init(bar_tempty + 8 * b, (kPair ? 2 : 1) * EPI_THREADS / 32);
+            mbar_init(bar_tempty + 8 * b, EPI_THREADS / 32);
         }
         mbar_init(bar_drain, 1);
         mbar_init(bar_epi, EPI_THREADS);
@@ -480,11 +498,24 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                         tma_load_2d(dB, &tmB, kb * BK, x.n0, fb);
                     } else if (kPair) {
                         // this CTA's 128 rows of A and 128 rows of B; both CTAs'
-                        // bytes complete on the leader's full barrier
+                        // bytes complete on the leader's full barrier.  B rows
+                        // 64h..64h+63 of this CTA feed column half h of the MMA:
+                        // SILU, tile rows 128 * rank + [0, 128) (the leader the
+                        // gate block, the peer the up block: each half gets 64
+                        // gate and the matching 64 up columns); otherwise tile
+                        // rows 128h + 64 * rank + [0, 64) (half h = output
+                        // columns 128h .. 128h + 127, in order)
                         const uint32_t lfb = lead_full + 8 * stage;
+                        const int brow = x.e * p.N + x.n0;
                         if (rank == 0) mbar_arrive_expect_tx(fb, 2 * STAGE_BYTES);
                         tma_load_2d_pair(dA, &tmA, kb * BK, x.m0, lfb);
-                        tma_load_2d_pair(dB, &tmB, kb * BK, x.e * p.N + x.n0 + (BN / 2) * (int)rank, lfb);
+                        if (kEpi == EPI_SILU) {
+                            tma_load_2d_pair(dB, &tmB, kb * BK, brow + BN_HALF * (int)rank, lfb);
+                        } else {
+                            tma_load_2d_pair(dB, &tmB, kb * BK, brow + 64 * (int)rank, lfb);
+                            tma_load_2d_pair(dB + L::B_BYTES / 2, &tmB, kb * BK, brow + BN_HALF + 64 * (int)rank,
+                                             lfb);
+                        }
                     } else {
                         mbar_arrive_expect_tx(fb, STAGE_BYTES);
                         tma_load_2d(dA, &tmA, kb * BK, x.m0, fb);
@@ -521,32 +552,54 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             for (int t = t_first; t < ntiles && ok; t += t_step) {
                 const Tile x = tile_of<kWgrad, kPair>(t, p, offs_s, pps_s, rank);
                 for (int kb = x.kb0; kb < x.kb1; ++kb) {
-                    if (!wait_bounded(bar_tempty + 8 * buf, bphase ^ 1, p.budget, abort_flag, p.status)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    if (!wait_bounded(bar_full + 8 * stage, phase, p.budget, abort_flag, p.status)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t aA = sbase + stage * STAGE_BYTES, aB = aA + A_BYTES;
-                    const uint32_t dtm = tmem_base + (uint32_t)(buf * BN);
                     if (kPair) {
+                        // two column halves, each into its own slot as soon as
+                        // that slot is free (the epilogue warpgroup of half 0
+                        // releases it while half 1's MMAs still run)
+                        if (!wait_bounded(bar_full + 8 * stage, phase, p.budget, abort_flag, p.status)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t aA = sbase + stage * STAGE_BYTES, aB = aA + A_BYTES;
 #pragma unroll
-                        for (int k4 = 0; k4 < BK / 32; ++k4)
-                            mma_f8_pair(dtm, sdesc(aA + 32 * k4), sdesc(aB + 32 * k4), k4 > 0 ? 1u : 0u);
-                        mma_commit_pair(bar_empty + 8 * stage);   // both CTAs' stage is free
-                        mma_commit_pair(bar_tfull + 8 * buf);     // both CTAs' epilogues may read
+                        for (int hh = 0; hh < 2; ++hh) {
+                            const int slot = 2 * buf + hh;
+                            if (!wait_bounded(bar_tempty + 8 * slot, bphase ^ 1, p.budget, abort_flag, p.status)) {
+                                ok = false;
+                                break;
+                            }
+                            tc_fence_after();
+                            const uint32_t dtm = tmem_base + (uint32_t)(buf * BN + hh * BN_HALF);
+                            const uint32_t bB = aB + (uint32_t)(hh * (L::B_BYTES / 2));
+#pragma unroll
+                            for (int k4 = 0; k4 < BK / 32; ++k4)
+                                mma_f8_pair(dtm, sdesc(aA + 32 * k4), sdesc(bB + 32 * k4), k4 > 0 ? 1u : 0u);
+                            mma_commit_pair(bar_tfull + 8 * slot);    // both CTAs' warpgroup hh may read
+                            issued = true;
+                        }
+                        if (!ok) break;
+                        mma_commit_pair(bar_empty + 8 * stage);       // both CTAs' stage is free
                     } else {
+                        if (!wait_bounded(bar_tempty + 8 * buf, bphase ^ 1, p.budget, abort_flag, p.status)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        if (!wait_bounded(bar_full + 8 * stage, phase, p.budget, abort_flag, p.status)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t aA = sbase + stage * STAGE_BYTES, aB = aA + A_BYTES;
+                        const uint32_t dtm = tmem_base + (uint32_t)(buf * BN);
 #pragma unroll
                         for (int k4 = 0; k4 < BK / 32; ++k4)
                             mma_f8(dtm, sdesc(aA + 32 * k4), sdesc(aB + 32 * k4), k4 > 0 ? 1u : 0u);
                         mma_commit(bar_empty + 8 * stage);
                         mma_commit(bar_tfull + 8 * buf);
+                        issued = true;
                     }
-                    issued = true;
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1;
@@ -587,14 +640,14 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             ephase ^= 1;
             return r;
         };
-        // SILU: the h codes of a tile are made during the next tile's K loop,
-        // four per thread after each K block (the scale is known by then).  The
-        // h values wait in this thread's own slot of a shared-memory staging
-        // area (2-SM layout) or in the bf16 h output the caller asked for
-        // (one-SM layout; read back one step ahead, from L2); without either
-        // the codes are made at once.
-        constexpr bool kDefer = kEpi == EPI_SILU;
-        const bool defer_on = kDefer && (kPair || p.out_bf16 != nullptr);
+        // SILU, 2-SM layout: the h codes of a tile are made during the next
+        // tile's K loop, four per thread after each K block (the scale is known
+        // by then); the h values wait in this thread's own slot of a
+        // shared-memory staging area.  (In the one-SM kernel the state this
+        // keeps live through the K loop cost register spills there that slowed
+        // it by a third; its codes are made at once.)
+        constexpr bool kDefer = kEpi == EPI_SILU && kPair;
+        constexpr bool defer_on = kDefer;
         int def_left = 0;           // h values of the deferred tile still to quantise
         float def_s = 0.0f;
         // the deferred tile's store coordinates (column, first row), per warp, kept in
@@ -682,37 +735,54 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     c_a = n_a, c_b0 = n_b0, c_b1 = n_b1;
                     if (kb + 2 < x.kb1) load_rows(kb + 2, n_a, n_b0, n_b1);
                 }
-                if (!warp_wait_bounded(bar_tfull + 8 * buf, bphase, p.budget, abort_flag, p.status)) {
+                const int slot = kPair ? 2 * buf + h : buf;   // this warpgroup's TMEM slot
+                if (!warp_wait_bounded(bar_tfull + 8 * slot, bphase, p.budget, abort_flag, p.status)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 const uint32_t cbase = lane_addr + (uint32_t)(buf * BN);
+                // TMEM column of chunk c (32 columns) of this warp's share: one
+                // SM, SILU: gate columns 64h.. then up columns 128 + 64h..; 2-SM:
+                // the warpgroup's own 128-column slot (SILU: 64 gate, 64 up)
                 auto col_of = [&](int c) -> uint32_t {
-                    if (kEpi == EPI_SILU) return (c < 2) ? (64 * h + 32 * c) : (128 + 64 * h + 32 * (c - 2));
+                    if (kEpi == EPI_SILU && !kPair) return (c < 2) ? (64 * h + 32 * c) : (128 + 64 * h + 32 * (c - 2));
                     return 128 * h + 32 * c;
                 };
-                // TMEM reads two chunks (64 columns) at a time with one wait per
-                // pair; the buffer goes back to the MMA as soon as the second
-                // pair has landed, before its FMAs
+                // The slot goes back to the MMA as soon as its last chunk has
+                // landed, before that chunk's FMAs.  TMEM reads: kAhead, one chunk
+                // ahead of the FMAs (chunk c + 1 in flight while chunk c is
+                // promoted); otherwise two chunks at a time, one wait per pair.
+                auto release = [&]() {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) {
+                        if (kPair)
+                            mbar_arrive_cluster(lead_tempty + 8 * slot);
+                        else
+                            mbar_arrive(bar_tempty + 8 * slot);
+                    }
+                };
                 uint32_t ra[32], rb[32];
+                if (kAhead) {
+                    MOE_TMEM_LD32(cbase + col_of(0), ra);
+                    tmem_wait_ld();
+                }
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     uint32_t *cur = (c & 1) ? rb : ra;
-                    if ((c & 1) == 0) {
+                    if (kAhead) {
+                        if (c < 3) {
+                            if (c & 1)
+                                MOE_TMEM_LD32(cbase + col_of(c + 1), ra);
+                            else
+                                MOE_TMEM_LD32(cbase + col_of(c + 1), rb);
+                        }
+                    } else if ((c & 1) == 0) {
                         MOE_TMEM_LD32(cbase + col_of(c), ra);
                         MOE_TMEM_LD32(cbase + col_of(c + 1), rb);
                         tmem_wait_ld();
-                        if (c == 2) {
-                            tc_fence_before();
-                            __syncwarp();
-                            if (lane == 0) {
-                                if (kPair)
-                                    mbar_arrive_cluster(lead_tempty + 8 * buf);
-                                else
-                                    mbar_arrive(bar_tempty + 8 * buf);
-                            }
-                        }
+                        if (c == 2) release();
                     }
                     if (kWgrad) {
                         // column scales of this chunk: 16-byte shared loads (a slot is
@@ -738,7 +808,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                             ffma2(acc[32 * c + i], acc[32 * c + i + 1], __uint_as_float(cur[i]),
                                   __uint_as_float(cur[i + 1]), sc, sc);
                     }
-
+                    if (kAhead && c < 3) {
+                        tmem_wait_ld();
+                        if (c == 2) release();
+                    }
                 }
                 if (kWgrad) {  // this warp has read the slot's scales
                     __syncwarp();
@@ -785,9 +858,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 const float s = block_scale(amax);
                 if (defer_on) {
                     while (def_left > 0) defer_step();   // a short tile: the previous codes first
-                    // the h row: to the staging slot, or to the caller's h output (written
-                    // now rather than below), then read back by the deferred steps
-                    uint8_t *dst = kPair ? hst : reinterpret_cast<uint8_t *>(p.out_bf16 + r * I + icol);
+                    // the h row to the staging slot, read back by the deferred steps
+                    uint8_t *dst = hst;
 #pragma unroll
                     for (int i0 = 0; i0 < 64; i0 += 8) *reinterpret_cast<uint4 *>(dst + 2 * i0) = pack8(&acc[i0]);
                     def_src = dst;
@@ -814,7 +886,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     }
                 }
                 if (h == 0) p.out_s[(int64_t)x.nt * p.R_cap + r] = s;
-                if (p.out_bf16 && !(defer_on && !kPair)) {   // (the one-SM deferral wrote it already)
+                if (p.out_bf16) {
                     uint16_t *hb = p.out_bf16 + r * I + icol;
 #pragma unroll
                     for (int i0 = 0; i0 < 64; i0 += 8) *reinterpret_cast<uint4 *>(hb + i0) = pack8(&acc[i0]);
@@ -948,17 +1020,18 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 // ------------------------------------------------------------------ host ----
 using namespace sm100;
 
-// 1-SM (0), 2-SM (1) or chosen per call (-1) for the rows-mode GEMMs.
+// Rows-mode GEMM kernel: 1-SM (0), 2-SM (1), 2-SM with TMEM reads one chunk
+// ahead (2), 1-SM with TMEM reads one chunk ahead (3), or chosen per call (-1).
 static int g_variant = 0;
 void set_gemm_variant(int v) { g_variant = v; }
 static int g_pair_clusters = 0;   // clusters of the last 2-SM launch
 int pair_clusters() { return g_pair_clusters; }
 
-template <int kEpi, bool kGather = false, bool kPair = false>
+template <int kEpi, bool kGather = false, bool kPair = false, bool kAhead = false>
 static int launch_one(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &c, const gemm::Args &args,
                       int grid, cudaStream_t s)
 {
-    auto kern = gemm::grouped_gemm_kernel<kEpi, kGather, kPair>;
+    auto kern = gemm::grouped_gemm_kernel<kEpi, kGather, kPair, kAhead>;
     constexpr int smem = gemm::smem_bytes<kEpi, kPair>();
     static bool configured = false;  // per process; attribute is per function
     if (!configured) {
@@ -1003,7 +1076,7 @@ static int launch_one(const CUtensorMap &a, const CUtensorMap &b, const CUtensor
 // those idle halves (at most one per segment) are a small share of the rows.
 static bool use_pair(int n_seg, int64_t R_cap)
 {
-    if (g_variant >= 0) return g_variant == 1;
+    if (g_variant >= 0) return g_variant == 1 || g_variant == 2;
     return (int64_t)n_seg * gemm::BM * 32 <= R_cap;
 }
 
@@ -1062,14 +1135,32 @@ int launch_grouped_gemm(int op, const moe_dims &d, int64_t R_cap, const int32_t 
     if (!ok) return MOE_ERR_CUDA;
     const int grid = sm_count();
     if (op != MOE_GEMM_WGRAD_DOWN && op != MOE_GEMM_WGRAD_GATEUP && use_pair(n_seg, R_cap)) {
-        // each CTA loads 128 rows of the 256-row B tile
+        // each CTA loads 128 rows of the 256-row B tile: one 128-row box (gate/up)
+        // or two 64-row boxes (the other GEMMs)
         const int64_t Kc = a.K, Nrows = (op == MOE_GEMM_GATEUP_SILU ? 2 * I : op == MOE_GEMM_DGRAD_DOWN_SILU ? I : D);
-        if (!make_map(&mB, g.b, Kc, E * Nrows, 128)) return MOE_ERR_CUDA;
+        if (!make_map(&mB, g.b, Kc, E * Nrows, op == MOE_GEMM_GATEUP_SILU ? 128 : 64)) return MOE_ERR_CUDA;
+        if (g_variant == 2) {
+            switch (op) {
+            case MOE_GEMM_GATEUP_SILU: return launch_one<gemm::EPI_SILU, false, true, true>(mA, mB, mC, a, grid, s);
+            case MOE_GEMM_DOWN:
+            case MOE_GEMM_DGRAD_GATEUP: return launch_one<gemm::EPI_BF16, false, true, true>(mA, mB, mC, a, grid, s);
+            default: return launch_one<gemm::EPI_DSILU, false, true, true>(mA, mB, mC, a, grid, s);
+            }
+        }
         switch (op) {
         case MOE_GEMM_GATEUP_SILU: return launch_one<gemm::EPI_SILU, false, true>(mA, mB, mC, a, grid, s);
         case MOE_GEMM_DOWN:
         case MOE_GEMM_DGRAD_GATEUP: return launch_one<gemm::EPI_BF16, false, true>(mA, mB, mC, a, grid, s);
         default: return launch_one<gemm::EPI_DSILU, false, true>(mA, mB, mC, a, grid, s);
+        }
+    }
+    if (g_variant == 3) {
+        switch (op) {
+        case MOE_GEMM_GATEUP_SILU: return launch_one<gemm::EPI_SILU, false, false, true>(mA, mB, mC, a, grid, s);
+        case MOE_GEMM_DOWN:
+        case MOE_GEMM_DGRAD_GATEUP: return launch_one<gemm::EPI_BF16, false, false, true>(mA, mB, mC, a, grid, s);
+        case MOE_GEMM_DGRAD_DOWN_SILU: return launch_one<gemm::EPI_DSILU, false, false, true>(mA, mB, mC, a, grid, s);
+        default: return launch_one<gemm::EPI_WGRAD, false, false, true>(mA, mB, mC, a, grid, s);
         }
     }
     switch (op) {

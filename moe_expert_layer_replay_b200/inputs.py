@@ -130,15 +130,17 @@ def _draw_routing(rng, wl: Workload, T: int) -> dict:
 
 
 def make_inputs(wl: Workload | str, seed: int = 0, T: int | None = None,
-                weights: bool = True, dy: bool | None = None) -> dict:
-    """Draw one workload's inputs.  ``T`` overrides the token count (for
-    small parity cases of the same recipe).  bf16 tensors come back as uint16
-    bit patterns; shapes: x [T, D], W_gate/W_up [E, I, D], W_down [E, D, I],
-    dy [T, D]."""
+                weights: bool = True, dy: bool | None = None, E: int | None = None) -> dict:
+    """Draw one workload's inputs.  ``T`` and ``E`` override the token and
+    expert counts (for small cases of the same recipe).  bf16 tensors come
+    back as uint16 bit patterns; shapes: x [T, D], W_gate/W_up [E, I, D],
+    W_down [E, D, I], dy [T, D]."""
     if isinstance(wl, str):
         wl = WORKLOADS[wl]
     if T is not None:
         wl = dataclasses.replace(wl, T=T)
+    if E is not None:
+        wl = dataclasses.replace(wl, E=E)
     rng = np.random.default_rng(seed)
     out = {"workload": wl}
     out.update(_draw_routing(rng, wl, wl.T))

@@ -1,6 +1,8 @@
-"""The 2-SM MMA variant of the rows-mode grouped GEMMs (tcgen05.mma
-cta_group::2: a pair of SMs per 256-row x 256-column tile, each CTA loading
-its own 128 rows of A and half of the weight tile) against the one-SM kernel:
+"""The other kernels of the rows-mode grouped GEMMs against the one-SM
+kernel: the 2-SM MMA (tcgen05.mma cta_group::2: a pair of SMs per 256-row x
+256-column tile, each CTA loading its own 128 rows of A and half of the
+weight tile, each K block issued as two 128-column halves), with either TMEM
+read order, and the one-SM kernel reading TMEM one chunk ahead:
 bit-identical h codes, scales, Y, d[g|u] and dX on the same operands (the two
 compute the same K-block partial products and promote them in the same
 order), including segments with an odd number of 128-row tiles (the idle half
@@ -29,7 +31,9 @@ CASES = {  # T, D, I, E, k, zipf (>= 2: three empty experts), train
     "odd_tiles_ragged": (1000, 512, 384, 8, 4, 1.0, True),
     "skew_empty": (700, 256, 256, 16, 4, 2.0, False),
     "shard_shape": (2048, 7168, 2048, 32, 8, 0.0, False),
+    "ragged_model_dim": (600, 384, 256, 8, 2, 0.5, True),   # a 128-column last tile in DOWN / DGRAD_GATEUP
 }
+VARIANTS = [1, 2, 3]
 
 
 def _run(A, variant, T, D, I, E, k, z, x, Wg, Wu, Wd, dy, train):
@@ -55,8 +59,9 @@ def _run(A, variant, T, D, I, E, k, z, x, Wg, Wu, Wd, dy, train):
     return out
 
 
+@pytest.mark.parametrize("variant", VARIANTS)
 @pytest.mark.parametrize("case", list(CASES))
-def test_pair_variant_equals_one_sm(A, case):
+def test_pair_variant_equals_one_sm(A, case, variant):
     T, D, I, E, k, zipf, train = CASES[case]
     rng = np.random.default_rng(400 + T)
     p = np.arange(1, E + 1, dtype=np.float64) ** -zipf
@@ -68,12 +73,13 @@ def test_pair_variant_equals_one_sm(A, case):
     Wg, Wu, Wd = rand_bf16(rng, (E, I, D), 0.02), rand_bf16(rng, (E, I, D), 0.02), rand_bf16(rng, (E, D, I), 0.02)
     dy = rand_bf16(rng, (T, D), 0.01)
     one = _run(A, 0, T, D, I, E, k, z, x, Wg, Wu, Wd, dy, train)
-    two = _run(A, 1, T, D, I, E, k, z, x, Wg, Wu, Wd, dy, train)
+    two = _run(A, variant, T, D, I, E, k, z, x, Wg, Wu, Wd, dy, train)
     for name in one:
-        same_bits(two[name], one[name], f"{name} (2-SM vs 1-SM)")
+        same_bits(two[name], one[name], f"{name} (variant {variant} vs 1-SM)")
 
 
-def test_pair_variant_segment_gemm(A):
+@pytest.mark.parametrize("variant", VARIANTS)
+def test_pair_variant_segment_gemm(A, variant):
     """Segments of an expert-parallel receiver, odd tile counts included."""
     rng = np.random.default_rng(410)
     E_loc, n_seg, D, I = 4, 8, 512, 256
@@ -88,8 +94,8 @@ def test_pair_variant_segment_gemm(A):
     xq = torch.from_numpy(rng.integers(0, 0x7F, (rows_cap, D), dtype=np.uint8)).cuda()
     xs = torch.from_numpy((rng.random((D // 128, rows_cap)) * 1e-2).astype(np.float32)).cuda()
     outs = []
-    for variant in (0, 1):
-        A.set_gemm_variant(variant)
+    for v in (0, variant):
+        A.set_gemm_variant(v)
         hq = torch.zeros(rows_cap, I, dtype=torch.uint8, device="cuda")
         hs = torch.zeros(I // 128, rows_cap, dtype=torch.float32, device="cuda")
         Y = torch.zeros(rows_cap, D, dtype=torch.bfloat16, device="cuda")
@@ -100,4 +106,4 @@ def test_pair_variant_segment_gemm(A):
         assert A.get_status() == A.OK
         outs.append((host(hq), host(hs), host(Y)))
     for a, b, name in zip(outs[0], outs[1], ["hq", "hs", "Y"]):
-        same_bits(b, a, f"{name} (2-SM vs 1-SM, segments)")
+        same_bits(b, a, f"{name} (variant {variant} vs 1-SM, segments)")
