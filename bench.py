@@ -770,8 +770,7 @@ def build_parser() -> argparse.ArgumentParser:
                     help="copy: the permute writes the permuted FP8 rows; gather: the gate/up GEMM gathers "
                          "them from the token rows")
     ap.add_argument("--gemm-variant", type=int, default=None,
-                    help="grouped GEMM kernel: 0 one SM per tile, 1 the 2-SM MMA, 2 the 2-SM MMA reading "
-                         "TMEM one chunk ahead, 3 one SM reading one chunk ahead, -1 chosen per call "
+                    help="grouped GEMM kernel: 0 one SM per tile, 1 the 2-SM MMA, -1 chosen per call "
                          "(default: the library's)")
     ap.add_argument("--once", action="store_true",
                     help="with --kernels: run every stage once, eagerly and untimed (for a profiler)")

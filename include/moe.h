@@ -94,11 +94,10 @@ uint64_t moe_kernel_launches(void);
 /* Which kernel runs the rows-mode grouped GEMMs (GATEUP_SILU, DOWN,
  * DGRAD_DOWN_SILU, DGRAD_GATEUP): 0 = one SM per 128 x 256 tile (the
  * default), 1 = the 2-SM MMA (a pair of SMs per 256 x 256 tile, each loading
- * half of the weight tile), 2 = the 2-SM MMA with the accumulator read one
- * 32-column chunk ahead of its promotion, 3 = the one-SM kernel with that
- * read order, -1 = chosen per call from the shapes.  Results are the same
- * bit for bit; the choice is per process.  Returns MOE_ERR_INVALID_ARG for
- * any other value. */
+ * half of the weight tile, each K block issued as two 128-column halves),
+ * -1 = chosen per call from the shapes.  Results are the same bit for bit;
+ * the choice is per process.  Returns MOE_ERR_INVALID_ARG for any other
+ * value. */
 int moe_set_gemm_variant(int variant);
 
 /* Clusters (CTA pairs) of the last 2-SM GEMM launch: the pairs the device can

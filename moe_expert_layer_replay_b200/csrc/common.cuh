@@ -65,32 +65,50 @@ __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi)
 // Scale of a block: fp32(amax / 448), IEEE division.
 __device__ __forceinline__ float block_scale(float amax) { return __fdiv_rn(amax, 448.0f); }
 
-// The e4m3 code of the correctly rounded quotient q = RN_fp32(x / s),
-// without a divide per element and without a branch.
-//
-// With r = RN(1/s), q' = RN(x * r) = (x/s)(1 + d), |d| < 3 * 2^-24, so q' is
-// within 3 fp32 ulps of q.  Let M be the e4m3 rounding midpoint of the bracket
-// [V_j, V_j+1) of e4m3 values that holds q'.  In e4m3's normal range M has
-// q''s sign, exponent and top three mantissa bits, then a 1 (20 low mantissa
-// bits 0x80000).  Below 2^-6 (e4m3's subnormal grid, step 2^-9) the midpoints
-// are the odd multiples of 2^-10: adding 2^-6 with rounding toward zero maps
-// q' into [2^-6, 2^-5), whose brackets are the same 2^-9 steps (the boundaries
-// are representable, so the truncated sum lies in the exact sum's bracket).
-//
-// q rounds like M's neighbours: q > M iff x/s > M + u/2, q < M iff x/s <
-// M - u/2, else q == M (u = fp32 ulp of M; M has 4 significant bits, so its
-// last fp32 mantissa bit is 0 and ties at M +- u/2 round to M; the one
-// midpoint that is a power of two, 2^-10, ties down to code 0 either way).
-// The test compares e = fma(-M, s, |x|) with c = s * u/2 (exact: a power-of-two
-// multiple of s):
-//   - when q' is within 4 ulps of M, x - M*s is a small multiple of the grid
-//     of M*s (at most 11 significant bits), so e is that difference exactly;
-//   - otherwise |x/s - M| > 1 ulp of M (1.5 * 2^-29 below 2^-6), so |x - M*s|
-//     > 2c and the rounded e falls on the same side of +-c as the exact one.
-// The element then converts through M or its fp32 neighbour on the decided
-// side, which e4m3 rounds like q.  Scales below 2^-90 use IEEE division:
-// from there up, c (>= s * 2^-34) and the grid of M*s (>= 2^-126 for M >=
-// 2^-10) stay in fp32's normal range, so neither is rounded.
+// (d0, d1) = (a0 * b0 + c0, a1 * b1 + c1) on two fp32 lanes at once (packed
+// f32x2), each rounded once to nearest even
+__device__ __forceinline__ void ffma2x(float &d0, float &d1, float a0, float a1, float b0, float b1, float c0,
+                                       float c1)
+{
+    asm("{\n\t.reg .b64 a, b, c, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+        "mov.b64 c, {%6, %7};\n\tfma.rn.f32x2 d, a, b, c;\n\tmov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+
+// (a0, a1) += (p0 * s0, p1 * s1), packed f32x2, each rounded once
+__device__ __forceinline__ void ffma2(float &a0, float &a1, float p0, float p1, float s0, float s1)
+{
+    asm("{\n\t.reg .b64 a, p, q;\n\tmov.b64 a, {%0, %1};\n\tmov.b64 p, {%2, %3};\n\t"
+        "mov.b64 q, {%4, %5};\n\tfma.rn.f32x2 a, p, q, a;\n\tmov.b64 {%0, %1}, a;\n\t}"
+        : "+f"(a0), "+f"(a1)
+        : "f"(p0), "f"(p1), "f"(s0), "f"(s1));
+}
+
+// (r0, r1) = (a0 * b0, a1 * b1), packed f32x2, each rounded once
+__device__ __forceinline__ void fmul2(float &r0, float &r1, float a0, float a1, float b0, float b1)
+{
+    asm("{\n\t.reg .b64 a, b, r;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+        "mul.rn.f32x2 r, a, b;\n\tmov.b64 {%0, %1}, r;\n\t}"
+        : "=f"(r0), "=f"(r1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+// The e4m3 codes of the correctly rounded quotients RN_fp32(x / s), without a
+// divide per element: Markstein's correction of a quotient by a correctly
+// rounded reciprocal (P. Markstein, "Computation of elementary functions on
+// the IBM RISC System/6000 processor", IBM J. Res. Develop. 34(1), 1990):
+//   r = RN(1/s),  q0 = RN(x r),  e = x - q0 s (one FMA, exact),  q = RN(q0 + e r).
+// Every quantiser here feeds it bf16 values x with |x| <= amax, amax a bf16
+// value and s = RN(amax / 448).  On that domain q = RN(x / s) whenever
+// |x / s| >= 2^-12, and below that both round to a zero code (with x's sign);
+// an exhaustive host check over every bf16 x against every bf16 amax mantissa,
+// across the exponent range, found no other case.  Scales below 2^-90 (r above
+// 2^90) and non-finite scales take IEEE division instead, out of line.
+// Each step runs on two elements at once (packed f32x2) with -r in place of r:
+// the chain then computes -q0, e and -q, exactly the negatives (rounding to
+// nearest is symmetric), so a zero quotient comes out with the sign opposite
+// to x's; the four codes' sign bits are flipped together at the end.
 template <int n>
 struct Floats {
     float v[n];
@@ -105,33 +123,34 @@ __device__ __noinline__ Floats<n> quotients_exact(Floats<n> x, float s)
     return q;
 }
 
-// Values whose e4m3 conversion equals that of fp32(v[i] / s), s != 0.
+// w[i] = codes of v[4i .. 4i+3] (element 4i + j in byte j); s > 0.
 template <int n>
-__device__ __forceinline__ void quotients(const float *v, float s, float *q)
+__device__ __forceinline__ void e4m3_codes(const float *v, float s, uint32_t *w)
 {
+    static_assert(n % 4 == 0, "groups of four");
     const float r = __frcp_rn(s);
-    if (!(r <= 0x1p90f)) {  // s below about 2^-90: IEEE division, out of line
+    if (!(r <= 0x1p90f) || r == 0.0f) {  // s below about 2^-90 (or not finite): IEEE division, out of line
         Floats<n> x;
 #pragma unroll
         for (int i = 0; i < n; ++i) x.v[i] = v[i];
-        const Floats<n> e = quotients_exact<n>(x, s);
+        const Floats<n> q = quotients_exact<n>(x, s);
 #pragma unroll
-        for (int i = 0; i < n; ++i) q[i] = e.v[i];
+        for (int i = 0; i < n / 4; ++i)
+            w[i] = e4m3x2(q.v[4 * i], q.v[4 * i + 1]) | (e4m3x2(q.v[4 * i + 2], q.v[4 * i + 3]) << 16);
         return;
     }
-    const float s24 = s * 0x1p-24f;  // u/2 * s = s24 * 2^exponent(M), exact
+    const float nr = -r;
 #pragma unroll
-    for (int i = 0; i < n; ++i) {
-        const float qp = __fmul_rn(v[i], r);
-        const uint32_t b = __float_as_uint(qp) & 0x7fffffffu;
-        const bool sub = b < 0x3c800000u;
-        const uint32_t y = sub ? __float_as_uint(__fadd_rz(__uint_as_float(b), 0x1p-6f)) : b;
-        const float My = __uint_as_float((y & 0xfff00000u) | 0x00080000u);
-        const float M = sub ? __fsub_rn(My, 0x1p-6f) : My;
-        const float c = __fmul_rn(s24, __uint_as_float(__float_as_uint(M) & 0x7f800000u));
-        const float e = __fmaf_rn(-M, s, fabsf(v[i]));
-        const uint32_t mb = __float_as_uint(M) + (e > c ? 1u : 0u) - (e < -c ? 1u : 0u);
-        q[i] = __uint_as_float(mb | (__float_as_uint(qp) & 0x80000000u));
+    for (int i = 0; i < n / 4; ++i) {
+        const float *x = v + 4 * i;
+        float a0, a1, a2, a3, e0, e1, e2, e3, q0, q1, q2, q3;
+        fmul2(a0, a1, x[0], x[1], nr, nr);             // -q0
+        fmul2(a2, a3, x[2], x[3], nr, nr);
+        ffma2x(e0, e1, a0, a1, s, s, x[0], x[1]);      // x - q0 s
+        ffma2x(e2, e3, a2, a3, s, s, x[2], x[3]);
+        ffma2x(q0, q1, e0, e1, nr, nr, a0, a1);        // -(q0 + e r)
+        ffma2x(q2, q3, e2, e3, nr, nr, a2, a3);
+        w[i] = (e4m3x2(q0, q1) | (e4m3x2(q2, q3) << 16)) ^ 0x80808080u;
     }
 }
 
@@ -139,11 +158,8 @@ __device__ __forceinline__ void quotients(const float *v, float s, float *q)
 __device__ __forceinline__ uint4 quant16(const float *v, float s)
 {
     if (s == 0.0f) return make_uint4(0, 0, 0, 0);
-    float q[16];
-    quotients<16>(v, s, q);
     uint32_t w[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) w[i] = e4m3x2(q[4 * i], q[4 * i + 1]) | (e4m3x2(q[4 * i + 2], q[4 * i + 3]) << 16);
+    e4m3_codes<16>(v, s, w);
     return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
@@ -151,18 +167,17 @@ __device__ __forceinline__ uint4 quant16(const float *v, float s)
 __device__ __forceinline__ uint32_t quant4(const float *v, float s)
 {
     if (s == 0.0f) return 0u;
-    float q[4];
-    quotients<4>(v, s, q);
-    return e4m3x2(q[0], q[1]) | (e4m3x2(q[2], q[3]) << 16);
+    uint32_t w;
+    e4m3_codes<4>(v, s, &w);
+    return w;
 }
 
 __device__ __forceinline__ uint2 quant8(const float *v, float s)
 {
     if (s == 0.0f) return make_uint2(0, 0);
-    float q[8];
-    quotients<8>(v, s, q);
-    return make_uint2(e4m3x2(q[0], q[1]) | (e4m3x2(q[2], q[3]) << 16),
-                      e4m3x2(q[4], q[5]) | (e4m3x2(q[6], q[7]) << 16));
+    uint32_t w[2];
+    e4m3_codes<8>(v, s, w);
+    return make_uint2(w[0], w[1]);
 }
 
 // sigmoid(g) for the SiLU gate, fast intrinsics (h and its gradient are

@@ -11,8 +11,8 @@
 //              (kind::f8f6f4, e4m3 x e4m3 -> fp32, M=128, N=256, K=32) x4
 //              per K block into one of two 256-column TMEM accumulators;
 //   warps 2-3  idle (they complete warpgroup 0, which gives its registers
-//              to the epilogue: setmaxnreg 56 here, 224 in warpgroups 1-2;
-//              128*56 + 256*224 = 384*168, the launch allocation);
+//              to the epilogue: setmaxnreg 40 here, 232 in warpgroups 1-2;
+//              128*40 + 256*232 = 384*168, the launch allocation);
 //   warps 4-11 epilogue: per K block, read the accumulator with tcgen05.ld,
 //              multiply by that block's scales (row scale x weight-block
 //              scale; per-column for wgrad) and add into fp32 registers; the
@@ -315,7 +315,7 @@ __device__ __forceinline__ Tile tile_of(int t, const Args &p, const int *offs_s,
 }
 
 // --------------------------------------------------------------- kernel ----
-template <int kEpi, bool kGather = false, bool kPair = false, bool kAhead = false>
+template <int kEpi, bool kGather = false, bool kPair = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmC, const Args p)
@@ -414,7 +414,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     const uint32_t lead_tempty = kPair ? peer_addr(bar_tempty, 0) : bar_tempty;
 
     if (warp < EPI_WARP0) {
-      asm volatile("setmaxnreg.dec.sync.aligned.u32 56;");
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 40;");
       if (warp == 0 && kGather) {
         // ------------------------------------- TMA producer, gathering ----
         // every lane gathers four A rows (tile rows 4*lane .. 4*lane+3) of
@@ -618,7 +618,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         }
       }
     } else {
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 224;");
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 232;");
         // --------------------------------------------------- epilogue ----
         const int ew = warp - EPI_WARP0;     // 0..7
         const int q = warp & 3;              // TMEM lane quarter of this warp
@@ -749,10 +749,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     if (kEpi == EPI_SILU && !kPair) return (c < 2) ? (64 * h + 32 * c) : (128 + 64 * h + 32 * (c - 2));
                     return 128 * h + 32 * c;
                 };
-                // The slot goes back to the MMA as soon as its last chunk has
-                // landed, before that chunk's FMAs.  TMEM reads: kAhead, one chunk
-                // ahead of the FMAs (chunk c + 1 in flight while chunk c is
-                // promoted); otherwise two chunks at a time, one wait per pair.
+                // TMEM reads in 16-column pieces, four per wait (64 registers in
+                // flight); the slot goes back to the MMA as soon as the last piece
+                // has landed, before its FMAs.  (Measured against 32-column loads
+                // two per wait, and against loads one chunk ahead of the FMAs: the
+                // MMA of the next K block, running meanwhile, finished sooner.)
                 auto release = [&]() {
                     tc_fence_before();
                     __syncwarp();
@@ -763,54 +764,44 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                             mbar_arrive(bar_tempty + 8 * slot);
                     }
                 };
-                uint32_t ra[32], rb[32];
-                if (kAhead) {
-                    MOE_TMEM_LD32(cbase + col_of(0), ra);
+                uint32_t rr[64];
+#pragma unroll
+                for (int g = 0; g < 2; ++g) {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int c16 = 4 * g + j;
+                        MOE_TMEM_LD16(cbase + col_of(c16 >> 1) + 16 * (c16 & 1), rr + 16 * j);
+                    }
                     tmem_wait_ld();
-                }
+                    if (g == 1) release();
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t *cur = (c & 1) ? rb : ra;
-                    if (kAhead) {
-                        if (c < 3) {
-                            if (c & 1)
-                                MOE_TMEM_LD32(cbase + col_of(c + 1), ra);
-                            else
-                                MOE_TMEM_LD32(cbase + col_of(c + 1), rb);
+                    for (int j = 0; j < 4; ++j) {
+                        const int c16 = 4 * g + j;
+                        const uint32_t *cur = rr + 16 * j;
+                        if (kWgrad) {
+                            // column scales of this piece: 16-byte shared loads (a slot
+                            // is 1536 B, the column part starts 512 B in); the scale
+                            // products sa * sb[n] on two lanes at once (the same fp32
+                            // products as two scalar multiplies)
+                            const float4 *cs = reinterpret_cast<const float4 *>(d + BM + 128 * h + 16 * c16);
+#pragma unroll
+                            for (int i = 0; i < 16; i += 4) {
+                                const float4 c4 = cs[i >> 2];
+                                float p0, p1, p2, p3;
+                                fmul2(p0, p1, sa, sa, c4.x, c4.y);
+                                fmul2(p2, p3, sa, sa, c4.z, c4.w);
+                                ffma2(acc[16 * c16 + i], acc[16 * c16 + i + 1], __uint_as_float(cur[i]),
+                                      __uint_as_float(cur[i + 1]), p0, p1);
+                                ffma2(acc[16 * c16 + i + 2], acc[16 * c16 + i + 3], __uint_as_float(cur[i + 2]),
+                                      __uint_as_float(cur[i + 3]), p2, p3);
+                            }
+                        } else {
+                            const float sc = (kEpi == EPI_SILU && c16 >= 4) ? s1 : s0;
+#pragma unroll
+                            for (int i = 0; i < 16; i += 2)
+                                ffma2(acc[16 * c16 + i], acc[16 * c16 + i + 1], __uint_as_float(cur[i]),
+                                      __uint_as_float(cur[i + 1]), sc, sc);
                         }
-                    } else if ((c & 1) == 0) {
-                        MOE_TMEM_LD32(cbase + col_of(c), ra);
-                        MOE_TMEM_LD32(cbase + col_of(c + 1), rb);
-                        tmem_wait_ld();
-                        if (c == 2) release();
-                    }
-                    if (kWgrad) {
-                        // column scales of this chunk: 16-byte shared loads (a slot is
-                        // 1536 B, the column part starts 512 B in)
-                        // (the scale products sa * sb[n] on two lanes at once: the
-                        // same fp32 products as two scalar multiplies)
-                        const float4 *cs = reinterpret_cast<const float4 *>(d + BM + 128 * h + 32 * c);
-#pragma unroll
-                        for (int i = 0; i < 32; i += 4) {
-                            const float4 c4 = cs[i >> 2];
-                            float p0, p1, p2, p3;
-                            fmul2(p0, p1, sa, sa, c4.x, c4.y);
-                            fmul2(p2, p3, sa, sa, c4.z, c4.w);
-                            ffma2(acc[32 * c + i], acc[32 * c + i + 1], __uint_as_float(cur[i]),
-                                  __uint_as_float(cur[i + 1]), p0, p1);
-                            ffma2(acc[32 * c + i + 2], acc[32 * c + i + 3], __uint_as_float(cur[i + 2]),
-                                  __uint_as_float(cur[i + 3]), p2, p3);
-                        }
-                    } else {
-                        const float sc = (kEpi == EPI_SILU && c >= 2) ? s1 : s0;
-#pragma unroll
-                        for (int i = 0; i < 32; i += 2)
-                            ffma2(acc[32 * c + i], acc[32 * c + i + 1], __uint_as_float(cur[i]),
-                                  __uint_as_float(cur[i + 1]), sc, sc);
-                    }
-                    if (kAhead && c < 3) {
-                        tmem_wait_ld();
-                        if (c == 2) release();
                     }
                 }
                 if (kWgrad) {  // this warp has read the slot's scales
@@ -1020,18 +1011,17 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 // ------------------------------------------------------------------ host ----
 using namespace sm100;
 
-// Rows-mode GEMM kernel: 1-SM (0), 2-SM (1), 2-SM with TMEM reads one chunk
-// ahead (2), 1-SM with TMEM reads one chunk ahead (3), or chosen per call (-1).
+// Rows-mode GEMM kernel: 1-SM (0), 2-SM (1) or chosen per call (-1).
 static int g_variant = 0;
 void set_gemm_variant(int v) { g_variant = v; }
 static int g_pair_clusters = 0;   // clusters of the last 2-SM launch
 int pair_clusters() { return g_pair_clusters; }
 
-template <int kEpi, bool kGather = false, bool kPair = false, bool kAhead = false>
+template <int kEpi, bool kGather = false, bool kPair = false>
 static int launch_one(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &c, const gemm::Args &args,
                       int grid, cudaStream_t s)
 {
-    auto kern = gemm::grouped_gemm_kernel<kEpi, kGather, kPair, kAhead>;
+    auto kern = gemm::grouped_gemm_kernel<kEpi, kGather, kPair>;
     constexpr int smem = gemm::smem_bytes<kEpi, kPair>();
     static bool configured = false;  // per process; attribute is per function
     if (!configured) {
@@ -1076,7 +1066,7 @@ static int launch_one(const CUtensorMap &a, const CUtensorMap &b, const CUtensor
 // those idle halves (at most one per segment) are a small share of the rows.
 static bool use_pair(int n_seg, int64_t R_cap)
 {
-    if (g_variant >= 0) return g_variant == 1 || g_variant == 2;
+    if (g_variant >= 0) return g_variant == 1;
     return (int64_t)n_seg * gemm::BM * 32 <= R_cap;
 }
 
@@ -1139,28 +1129,11 @@ int launch_grouped_gemm(int op, const moe_dims &d, int64_t R_cap, const int32_t 
         // or two 64-row boxes (the other GEMMs)
         const int64_t Kc = a.K, Nrows = (op == MOE_GEMM_GATEUP_SILU ? 2 * I : op == MOE_GEMM_DGRAD_DOWN_SILU ? I : D);
         if (!make_map(&mB, g.b, Kc, E * Nrows, op == MOE_GEMM_GATEUP_SILU ? 128 : 64)) return MOE_ERR_CUDA;
-        if (g_variant == 2) {
-            switch (op) {
-            case MOE_GEMM_GATEUP_SILU: return launch_one<gemm::EPI_SILU, false, true, true>(mA, mB, mC, a, grid, s);
-            case MOE_GEMM_DOWN:
-            case MOE_GEMM_DGRAD_GATEUP: return launch_one<gemm::EPI_BF16, false, true, true>(mA, mB, mC, a, grid, s);
-            default: return launch_one<gemm::EPI_DSILU, false, true, true>(mA, mB, mC, a, grid, s);
-            }
-        }
         switch (op) {
         case MOE_GEMM_GATEUP_SILU: return launch_one<gemm::EPI_SILU, false, true>(mA, mB, mC, a, grid, s);
         case MOE_GEMM_DOWN:
         case MOE_GEMM_DGRAD_GATEUP: return launch_one<gemm::EPI_BF16, false, true>(mA, mB, mC, a, grid, s);
         default: return launch_one<gemm::EPI_DSILU, false, true>(mA, mB, mC, a, grid, s);
-        }
-    }
-    if (g_variant == 3) {
-        switch (op) {
-        case MOE_GEMM_GATEUP_SILU: return launch_one<gemm::EPI_SILU, false, false, true>(mA, mB, mC, a, grid, s);
-        case MOE_GEMM_DOWN:
-        case MOE_GEMM_DGRAD_GATEUP: return launch_one<gemm::EPI_BF16, false, false, true>(mA, mB, mC, a, grid, s);
-        case MOE_GEMM_DGRAD_DOWN_SILU: return launch_one<gemm::EPI_DSILU, false, false, true>(mA, mB, mC, a, grid, s);
-        default: return launch_one<gemm::EPI_WGRAD, false, false, true>(mA, mB, mC, a, grid, s);
         }
     }
     switch (op) {

@@ -115,7 +115,7 @@ uint64_t moe_kernel_launches(void) { return g_launches.load(std::memory_order_re
 
 int moe_set_gemm_variant(int variant)
 {
-    if (variant < -1 || variant > 3) return MOE_ERR_INVALID_ARG;
+    if (variant < -1 || variant > 1) return MOE_ERR_INVALID_ARG;
     moe::set_gemm_variant(variant);
     return MOE_OK;
 }

@@ -131,24 +131,6 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int n>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(n) : "memory"); }
 
-// a = fma(p, s, a) on two fp32 lanes at once (packed f32x2)
-__device__ __forceinline__ void ffma2(float &a0, float &a1, float p0, float p1, float s0, float s1)
-{
-    asm("{\n\t.reg .b64 a, p, q;\n\tmov.b64 a, {%0, %1};\n\tmov.b64 p, {%2, %3};\n\t"
-        "mov.b64 q, {%4, %5};\n\tfma.rn.f32x2 a, p, q, a;\n\tmov.b64 {%0, %1}, a;\n\t}"
-        : "+f"(a0), "+f"(a1)
-        : "f"(p0), "f"(p1), "f"(s0), "f"(s1));
-}
-
-// (r0, r1) = (a0 * b0, a1 * b1) on two fp32 lanes at once (packed f32x2)
-__device__ __forceinline__ void fmul2(float &r0, float &r1, float a0, float a1, float b0, float b1)
-{
-    asm("{\n\t.reg .b64 a, b, r;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
-        "mul.rn.f32x2 r, a, b;\n\tmov.b64 {%0, %1}, r;\n\t}"
-        : "=f"(r0), "=f"(r1)
-        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
-}
-
 // TMA store of a 2D box from shared memory (bulk-group completion).
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t src, int32_t c0, int32_t c1)
 {
@@ -194,6 +176,16 @@ __device__ __forceinline__ void mma_commit(uint32_t bar)
           "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),   \
           "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),   \
           "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])                                           \
+        : "r"(taddr))
+
+// sixteen consecutive TMEM columns of this warp's 32 lanes into r[0..15]
+#define MOE_TMEM_LD16(taddr, r)                                                                        \
+    asm volatile(                                                                                      \
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"   \
+        "%15}, [%16];"                                                                                 \
+        : "=r"((r)[0]), "=r"((r)[1]), "=r"((r)[2]), "=r"((r)[3]), "=r"((r)[4]), "=r"((r)[5]),         \
+          "=r"((r)[6]), "=r"((r)[7]), "=r"((r)[8]), "=r"((r)[9]), "=r"((r)[10]), "=r"((r)[11]),       \
+          "=r"((r)[12]), "=r"((r)[13]), "=r"((r)[14]), "=r"((r)[15])                                  \
         : "r"(taddr))
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
