@@ -125,62 +125,118 @@ int launch_dispatch_quant(const uint16_t *x, int64_t T, int64_t D, const int32_t
 // Row r of the source is in[r*ld], or, when src_idx != nullptr, the token row
 // in[(src_idx[r]/k)*ld] (a zero row for src_idx[r] < 0): the gather that
 // makes the permuted activation rows without materialising them.
-// Block = 128 rows x 64 columns; 256 threads: thread (col = tid%64,
-// part = tid/64) reduces 32 rows of its column and writes 32 codes.
+// Tiles of 128 rows x 64 columns; a persistent grid sized to the blocks the
+// SMs hold at once.  Each block keeps the copies of its next two tiles in
+// flight (cp.async into a three-slot ring in shared memory, 16 bytes a copy,
+// zero-filled for missing rows) while it quantises the current one.  256
+// threads: thread (col = tid%64, part = tid/64) reduces 32 rows of its column
+// and writes 32 codes.  Row blocks vary fastest, so the blocks in flight
+// share their column block: their codes fill whole lines of the transposed
+// output, and, gathering, the token rows they read stay in L2 for the k
+// permuted rows that repeat them.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) quant_rows128_kernel(const uint16_t *__restrict__ in, int64_t ld,
+constexpr int kR128Pad = 72;   // bf16 per tile row: 144 B, 16-byte aligned rows
+constexpr int kR128Slots = 3;
+constexpr int kR128Smem = kR128Slots * 128 * kR128Pad * 2;
+
+__device__ __forceinline__ void cp_async16_zfill(void *dst, const void *src, uint32_t bytes)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(
+                     static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+                 "l"(src), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit_group() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int n>
+__device__ __forceinline__ void cp_async_wait_groups() { asm volatile("cp.async.wait_group %0;" ::"n"(n) : "memory"); }
+
+__global__ void __launch_bounds__(256, 4) quant_rows128_kernel(const uint16_t *__restrict__ in, int64_t ld,
                                                             const int32_t *__restrict__ src_idx, int k,
                                                             int64_t rows, int64_t cols, int64_t ld_rows,
                                                             uint8_t *__restrict__ qT,
                                                             float *__restrict__ sT)
 {
-    // bf16 tile, rows of 64 columns + 8 pad (144 B: 16-byte aligned rows, and a
-    // warp's 32 consecutive columns of one row are 64 contiguous bytes)
-    __shared__ __align__(16) uint16_t tile[128][72];
+    extern __shared__ __align__(16) uint16_t ring[];   // [kR128Slots][128][kR128Pad]
     __shared__ float part_max[4][64];
     const int tid = threadIdx.x;
-    const int64_t r0 = (int64_t)blockIdx.x * 128;
-    const int64_t c0 = (int64_t)blockIdx.y * 64;
+    const int64_t ntr = (rows + 127) / 128, ntiles = ntr * ((cols + 63) / 64);
+    // the source row of each of this thread's four pieces of tile t (-1: zeros);
+    // gathering, the indices are loaded one tile ahead of their copies, so the
+    // copies never wait for them
+    auto rows_of = [&](int64_t t, int32_t *src_row) {
 #pragma unroll
-    for (int it = 0; it < 4; ++it) {
-        int idx = it * 256 + tid;  // 1024 16-byte pieces: 128 rows x 8
-        int r = idx >> 3, cc = (idx & 7) * 8;
-        int64_t gr = r0 + r;
-        const uint16_t *src = nullptr;
-        if (gr < rows) {
-            if (src_idx) {
-                int si = src_idx[gr];
-                if (si >= 0) src = in + (int64_t)(si / k) * ld;
-            } else {
-                src = in + gr * ld;
+        for (int it = 0; it < 4; ++it) {
+            const int64_t gr = (t % ntr) * 128 + ((it * 256 + tid) >> 3);
+            int32_t sr = -1;
+            if (t < ntiles && gr < rows) {
+                if (src_idx) {
+                    const int si = src_idx[gr];
+                    sr = si >= 0 ? si / k : -1;
+                } else {
+                    sr = (int32_t)gr;
+                }
+            }
+            src_row[it] = sr;
+        }
+    };
+    // the copies of tile t into ring slot `slot` (one commit group; none past the end)
+    auto issue = [&](int64_t t, int slot, const int32_t *src_row) {
+        if (t < ntiles) {
+            const int64_t c0 = (t / ntr) * 64;
+            uint16_t *tile = ring + slot * 128 * kR128Pad;
+#pragma unroll
+            for (int it = 0; it < 4; ++it) {
+                const int idx = it * 256 + tid;  // 1024 16-byte pieces: 128 rows x 8
+                const int r = idx >> 3, cc = (idx & 7) * 8;
+                const bool ok = src_row[it] >= 0 && c0 + cc < cols;
+                // (no bytes are read from the base address when zero-filling)
+                cp_async16_zfill(tile + r * kR128Pad + cc, ok ? in + (int64_t)src_row[it] * ld + c0 + cc : in,
+                                 ok ? 16u : 0u);
             }
         }
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (src && c0 + cc < cols) v = *reinterpret_cast<const uint4 *>(src + c0 + cc);
-        *reinterpret_cast<uint4 *>(&tile[r][cc]) = v;
-    }
-    __syncthreads();
-    const int col = tid & 63, part = tid >> 6;
-    float v[32];  // this thread's 32 rows of its column
-    float amax = 0.0f;
+        cp_async_commit_group();   // (an empty group past the end keeps the count)
+    };
+    const int64_t G = gridDim.x;
+    int slot = 0;
+    int32_t rw[4], nxt[4];
+    rows_of(blockIdx.x, rw);
+    issue(blockIdx.x, 0, rw);
+    rows_of(blockIdx.x + G, rw);
+    issue(blockIdx.x + G, 1, rw);
+    rows_of(blockIdx.x + 2 * G, nxt);
+    for (int64_t t = blockIdx.x; t < ntiles; t += G) {
+        issue(t + 2 * G, (slot + 2) % kR128Slots, nxt);
+        rows_of(t + 3 * G, nxt);
+        cp_async_wait_groups<2>();   // tile t has landed
+        __syncthreads();
+        const uint16_t *tile = ring + slot * 128 * kR128Pad;
+        const int64_t r0 = (t % ntr) * 128, c0 = (t / ntr) * 64;
+        const int col = tid & 63, part = tid >> 6;
+        float v[32];  // this thread's 32 rows of its column
+        float amax = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        v[i] = __uint_as_float((uint32_t)tile[part * 32 + i][col] << 16);
-        amax = fmaxf(amax, fabsf(v[i]));
-    }
-    part_max[part][col] = amax;
-    __syncthreads();
-    amax = fmaxf(fmaxf(part_max[0][col], part_max[1][col]), fmaxf(part_max[2][col], part_max[3][col]));
-    const float s = block_scale(amax);
-    const int64_t gc = c0 + col;
-    if (gc >= cols) return;
+        for (int i = 0; i < 32; ++i) {
+            v[i] = __uint_as_float((uint32_t)tile[(part * 32 + i) * kR128Pad + col] << 16);
+            amax = fmaxf(amax, fabsf(v[i]));
+        }
+        part_max[part][col] = amax;
+        __syncthreads();
+        amax = fmaxf(fmaxf(part_max[0][col], part_max[1][col]), fmaxf(part_max[2][col], part_max[3][col]));
+        const float s = block_scale(amax);
+        const int64_t gc = c0 + col;
+        if (gc < cols) {
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const int64_t rr = r0 + part * 32 + h * 16;
-        const uint4 codes = quant16(v + 16 * h, s);
-        if (rr < rows) *reinterpret_cast<uint4 *>(qT + gc * ld_rows + rr) = codes;
+            for (int h = 0; h < 2; ++h) {
+                const int64_t rr = r0 + part * 32 + h * 16;
+                const uint4 codes = quant16(v + 16 * h, s);
+                if (rr < rows) *reinterpret_cast<uint4 *>(qT + gc * ld_rows + rr) = codes;
+            }
+            if (part == 0) sT[(r0 / 128) * cols + gc] = s;
+        }
+        __syncthreads();  // this slot and part_max are read before they are refilled
+        slot = (slot + 1) % kR128Slots;
     }
-    if (part == 0) sT[(r0 / 128) * cols + gc] = s;
+    cp_async_wait_groups<0>();   // (only empty groups remain; none outlives the block)
 }
 
 int launch_quant_rows128(const uint16_t *in, int64_t ld, const int32_t *src_idx, int k,
@@ -188,8 +244,22 @@ int launch_quant_rows128(const uint16_t *in, int64_t ld, const int32_t *src_idx,
                          cudaStream_t s)
 {
     if (rows == 0 || cols == 0) return MOE_OK;
-    dim3 grid((unsigned)((rows + 127) / 128), (unsigned)((cols + 63) / 64));
-    quant_rows128_kernel<<<grid, 256, 0, s>>>(in, ld, src_idx, k, rows, cols, ld_rows, qT, sT);
+    if (rows > INT32_MAX) return MOE_ERR_UNSUPPORTED;   // row indices are 32-bit in the kernel
+    static int per_sm = 0, sms = 0;   // per process: the device and the kernel's resources are fixed
+    if (per_sm == 0) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaFuncSetAttribute(quant_rows128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kR128Smem) !=
+                cudaSuccess ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quant_rows128_kernel, 256, kR128Smem) !=
+                cudaSuccess ||
+            per_sm <= 0)
+            return MOE_ERR_CUDA;
+    }
+    const int64_t ntiles = ((rows + 127) / 128) * ((cols + 63) / 64);
+    const int64_t grid = ntiles < (int64_t)per_sm * sms ? ntiles : (int64_t)per_sm * sms;
+    quant_rows128_kernel<<<(unsigned)grid, 256, kR128Smem, s>>>(in, ld, src_idx, k, rows, cols, ld_rows, qT, sT);
     count_launch();
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
@@ -235,6 +305,9 @@ int launch_pad_rows(const int32_t *counts, const int32_t *offsets, int E, int64_
 // 128x128 blocks of a stack of matrices in[e] = in + e*in_expert_stride,
 // [rows][cols] with row stride ld.  One block per (column block, row block,
 // expert); 256 threads, each converting 8 contiguous elements of 8 rows.
+// The block is staged in shared memory by cp.async (no values held in
+// registers while the copies fly), so several blocks per SM keep copies in
+// flight.
 // Output row block of source row block rb is rb*rb_mul + rb_add (this lays
 // gate and up out interleaved by 128-row blocks).
 //   q  [e]: codes at (dst row, c), row stride cols;
@@ -248,26 +321,36 @@ __global__ void __launch_bounds__(256) quant_128x128_kernel(
     int64_t s_es, uint8_t *__restrict__ qT, int64_t qT_ld, int64_t qT_es, float *__restrict__ sT,
     int64_t sT_ld, int64_t sT_es)
 {
+    // the bf16 block (rows of 136: 272 B, 16-byte aligned), later reused for
+    // its codes (rows of 144 B) once every thread holds its own in registers
+    __shared__ __align__(16) uint16_t tile[128][136];
     __shared__ float warp_max[8];
-    __shared__ uint8_t codes_s[128][144];
+    uint8_t(*codes_s)[144] = reinterpret_cast<uint8_t(*)[144]>(&tile[0][0]);
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const int64_t cb = blockIdx.x, rb = blockIdx.y, e = blockIdx.z;
     const int64_t nbc = (cols + 127) / 128;
     const uint16_t *src = in + e * in_es;
+    // the whole block into shared memory at once: eight 16-byte copies per
+    // thread in flight, none held in registers (zero-filled past the edges)
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+        const int idx = it * 256 + tid;  // 2048 pieces: 128 rows x 16
+        const int r = idx >> 4, c = (idx & 15) * 8;
+        const int64_t gr = rb * 128 + r, gc = cb * 128 + c;
+        const bool in_range = gr < rows && gc < cols;
+        cp_async16_zfill(&tile[r][c], in_range ? src + gr * ld + gc : src, in_range ? 16u : 0u);
+    }
+    cp_async_commit_group();
+    cp_async_wait_groups<0>();
+    __syncthreads();
     const int cc = (tid & 15) * 8;   // column within the block
     const int rr0 = tid >> 4;        // rows rr0, rr0+16, ...
-    float v[8][8];
     float amax = 0.0f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        int64_t r = rb * 128 + rr0 + 16 * i, c = cb * 128 + cc;
-        if (r < rows && c < cols) {
-            unpack8(*reinterpret_cast<const uint4 *>(src + r * ld + c), v[i]);
-        } else {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) v[i][j] = 0.0f;
-        }
-        amax = absmax8(v[i], amax);
+        float v[8];
+        unpack8(*reinterpret_cast<const uint4 *>(&tile[rr0 + 16 * i][cc]), v);
+        amax = absmax8(v, amax);
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, off));
@@ -279,15 +362,20 @@ __global__ void __launch_bounds__(256) quant_128x128_kernel(
     const float s = block_scale(amax);
     const int64_t drb = rb * rb_mul + rb_add;
     uint8_t *qe = q + e * q_es;
+    uint2 c8[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        uint2 c8 = quant8(v[i], s);
-        int64_t r = rb * 128 + rr0 + 16 * i, c = cb * 128 + cc;
-        if (r < rows && c < cols) *reinterpret_cast<uint2 *>(qe + (drb * 128 + rr0 + 16 * i) * cols + c) = c8;
-        *reinterpret_cast<uint2 *>(&codes_s[rr0 + 16 * i][cc]) = c8;
+        float v[8];
+        unpack8(*reinterpret_cast<const uint4 *>(&tile[rr0 + 16 * i][cc]), v);
+        c8[i] = quant8(v, s);
+        const int64_t r = rb * 128 + rr0 + 16 * i, c = cb * 128 + cc;
+        if (r < rows && c < cols) *reinterpret_cast<uint2 *>(qe + (drb * 128 + rr0 + 16 * i) * cols + c) = c8[i];
     }
     if (tid == 0) sc[e * s_es + drb * nbc + cb] = s;
     if (!qT) return;
+    __syncthreads();   // every thread has read its bf16 values: the tile takes the codes
+#pragma unroll
+    for (int i = 0; i < 8; ++i) *reinterpret_cast<uint2 *>(&codes_s[rr0 + 16 * i][cc]) = c8[i];
     __syncthreads();
     // transposed: tile column c -> 128 bytes of qT row (cb*128 + c); each
     // thread assembles 16 codes (rows 16*h .. 16*h+15) of one column.  A warp
