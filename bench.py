@@ -45,6 +45,7 @@ if ROOT not in sys.path:
 METRIC = "MoE-layer tokens/s; grouped FP8 GEMM TFLOP/s as % of dense FP8 peak"
 UNIT = "tokens/s"
 FP8_OVER_BF16 = 2.0  # nominal dense ratio (4.5 / 2.25 PFLOP/s), used only when no FP8 peak was measured
+FP4_OVER_FP8 = 2.0   # nominal dense ratio (9 / 4.5 PFLOP/s): the FP4 peak is this times the measured FP8 peak
 
 # DRAM traffic (read + write bytes) of one gate/up GEMM launch per workload,
 # from an ncu capture of dram__bytes_read.sum + dram__bytes_write.sum on that
@@ -597,6 +598,42 @@ def e2e_run(args, wl, d, W, inp, world, barrier, gather=False):
     return val, h2d, d2h
 
 
+def nvfp4_stages(abi, d, B, x, wg, wu, R_pad):
+    """The NVFP4 variant of the gate/up GEMM (f4) as extra report stages: the
+    permuted rows of x and each expert's [W_gate; W_up] quantised to NVFP4
+    (scales in the block-scaled MMA's layout), then the grouped NVFP4 GEMM
+    with fp32 output.  The permuted bf16 rows are gathered by torch once,
+    outside the timed stages (input preparation only)."""
+    import torch
+    D, I, E = d.D, d.I, d.E
+    R_cap = B.R_cap
+    src = B.src[:R_cap].long()
+    rows = torch.zeros(R_cap, D, dtype=torch.bfloat16, device="cuda")
+    ok = src >= 0
+    rows[ok] = x[src[ok] // d.k]
+    wgu = torch.cat([wg, wu], dim=1).contiguous()          # [E][2I][D]
+    q = torch.empty(R_cap, D // 2, dtype=torch.uint8, device="cuda")
+    sf = torch.empty(R_cap * D // 16, dtype=torch.uint8, device="cuda")
+    amax = torch.empty(1, device="cuda")
+    sg = torch.empty(1, device="cuda")
+    wq = torch.empty(E, 2 * I, D // 2, dtype=torch.uint8, device="cuda")
+    wsf = torch.empty(E, 2 * I * D // 16, dtype=torch.uint8, device="cuda")
+    wamax = torch.empty(E, device="cuda")
+    wsg = torch.empty(E, device="cuda")
+    for e in range(E):
+        abi.quant_nvfp4(wgu[e], 2 * I, D, D, wq[e], wsf[e], wamax[e:e + 1], wsg[e:e + 1],
+                        sf_layout=abi.NVFP4_SF_MMA)
+    out = torch.empty(R_cap, 2 * I, dtype=torch.float32, device="cuda")
+    return [
+        ("NVFP4 quant of the permuted rows", lambda: abi.quant_nvfp4(rows, R_cap, D, D, q, sf, amax, sg,
+                                                                      sf_layout=abi.NVFP4_SF_MMA),
+         "B", 2 * 2 * R_cap * D + R_cap * (D // 2 + D // 16)),
+        ("gemm gate/up NVFP4 (fp32 out)", lambda: abi.gemm_nvfp4(R_cap, 2 * I, D, E, B.offsets, q, sf, sg, wq, wsf,
+                                                                  wsg, out),
+         "F4", 4.0 * d.T * d.k * D * I),
+    ]
+
+
 def run_kernels(args, names):
     """Per-stage device time of one layer pass for each named workload (the
     stages of the hot path, forward and, for the training workload, backward):
@@ -668,6 +705,8 @@ def run_kernels(args, names):
                 d, B.offsets, B.src, B.xq_tok, B.xs_tok, W.wgu_q, W.wgu_s, out_q=B.hq, out_s=B.hs), "F",
              4.0 * R * D * I),
         ]
+        if not args.once and D % 256 == 0:
+            st += nvfp4_stages(abi, d, B, x, wg, wu, R_pad)
         if train:
             dy = bfd(inp["dy"])
             st += [
@@ -730,10 +769,13 @@ def run_kernels(args, names):
                 ts.append(e0.elapsed_time(e1) / n)
             del g
             ms = statistics.median(ts)
-            if kind == "F":
+            if kind in ("F", "F4"):
                 ach = units / (ms * 1e-3) / 1e12
+                pk = fp8 * (FP4_OVER_FP8 if kind == "F4" else 1.0)
                 out.append({"stage": sname, "us": round(ms * 1e3, 2), "flop": units, "tflops": round(ach, 1),
-                            "frac": round(ach / fp8, 4)})
+                            "frac": round(ach / pk, 4)})
+                if kind == "F4":
+                    out[-1]["peak_note"] = "dense FP4 = 2 x the measured FP8 peak (nominal 9 vs 4.5 PFLOP/s)"
             else:
                 ach = units / (ms * 1e-3) / 1e9
                 out.append({"stage": sname, "us": round(ms * 1e3, 2), "bytes": units, "gbs": round(ach, 1),
@@ -742,7 +784,7 @@ def run_kernels(args, names):
         if abi.get_status() != abi.OK:
             raise RuntimeError("device status after the timed replays")
         # (the gathered gate/up GEMM is an alternative to the copy path's, not an extra step)
-        gf = [o for o in out if "flop" in o and "gathering" not in o["stage"]]
+        gf = [o for o in out if "flop" in o and "gathering" not in o["stage"] and "NVFP4" not in o["stage"]]
         line = {"kernels_report": _workload_desc(wl), "R": R, "R_pad": R_pad,
                 "gemm_pair_clusters": abi.gemm_pair_clusters(),
                 "peaks": {"hbm_gbs": hbm, "hbm_source": src, "fp8_tflops": fp8, "fp8_source": fp8_src},

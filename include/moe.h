@@ -229,15 +229,44 @@ int moe_quant_fp8_block(const uint16_t *in, int64_t rows, int64_t cols, int64_t 
  * ld % 8 == 0, cols % 16 == 0, in 16-byte aligned, q 8-byte aligned):
  *   amax (one float)  max |x| over the tensor;
  *   s_g  (one float)  tensor scale fp32(2688 / amax) (1 if amax = 0);
- *   sf [rows][cols/16] e4m3 block-scale codes: e4m3(RNE, satfinite)(
- *                     fp32(fp32(amax_b / 6) * s_g)), amax_b over 16 elements;
+ *   sf                e4m3 block-scale codes e4m3(RNE, satfinite)(
+ *                     fp32(fp32(amax_b / 6) * s_g)), amax_b over 16 elements,
+ *                     laid out by sf_layout:
+ *                       MOE_NVFP4_SF_ROWS  [rows][cols/16];
+ *                       MOE_NVFP4_SF_MMA   the block-scaled MMA's layout
+ *                         (rows % 128 == 0, cols % 64 == 0): 512-byte atoms,
+ *                         atom (rb, ks) of 128-row block rb and 64-column step
+ *                         ks at (rb * cols/64 + ks) * 512; inside it the scale
+ *                         of row 128 rb + 32 r1 + r0, group 4 ks + j at byte
+ *                         16 r0 + 4 r1 + j;
  *   q  [rows][cols/2] e2m1 codes, two per byte (element 2i in the low
  *                     nibble): 0 where the block scale is 0, else e2m1(RNE,
  *                     satfinite)(fp32(x * fp32(s_g / value(sf)))).
  * Value of an element: e2m1(q) * value(sf) / s_g.  amax and s_g are device
- * words the call writes (amax is zeroed first, then accumulated). */
+ * words the call writes (amax is zeroed first, then accumulated).
+ * MOE_ERR_INVALID_ARG for an unknown layout or shapes the layout excludes. */
+#define MOE_NVFP4_SF_ROWS 0
+#define MOE_NVFP4_SF_MMA 1
 int moe_quant_nvfp4(const uint16_t *in, int64_t rows, int64_t cols, int64_t ld, uint8_t *q, uint8_t *sf,
-                    float *amax, float *s_g, void *stream);
+                    int32_t sf_layout, float *amax, float *s_g, void *stream);
+
+/* NVFP4 grouped GEMM [P4 §Future work: NVFP4 on Blackwell], on the tensor
+ * cores' block-scaled MMA (kind::mxf4nvf4, 16-element ue4m3 scales):
+ *   out[r][n] = sum_k value(A)[r][k] * value(B_e)[n][k]   for r in segment e,
+ * segments [offsets[e], offsets[e+1]) of the rows, 128-aligned (n_seg <= 256;
+ * offsets on the device, read there).  Operands as moe_quant_nvfp4 makes
+ * them with MOE_NVFP4_SF_MMA:
+ *   a    [rows_cap][K/2] packed e2m1 codes;   sfa  scale atoms of A (rows_cap rows);
+ *   a_sg A's tensor scale (device float);
+ *   b    [n_seg][N][K/2] codes of each segment's B;  sfb  their atoms (n_seg * N rows);
+ *   b_sg [n_seg] tensor scales of the B's (device);
+ *   out  [rows_cap][N] fp32, rows past offsets[n_seg] untouched.
+ * N % 256 == 0, K % 256 == 0, rows_cap % 128 == 0; pointers 16-byte aligned
+ * (MOE_ERR_INVALID_ARG otherwise).  The accumulation is fp32 over exact
+ * products; the result is scaled by 1 / (a_sg * b_sg[e]). */
+int moe_gemm_nvfp4(int64_t rows_cap, int32_t N, int32_t K, int32_t n_seg, const int32_t *offsets,
+                   const uint8_t *a, const uint8_t *sfa, const float *a_sg, const uint8_t *b, const uint8_t *sfb,
+                   const float *b_sg, float *out, void *stream);
 
 /* Expert weights (a5): 128x128 FP8 of W_gate, W_up [E][I][D] and W_down [E][D][I].
  *   wgu_q [E][2I][D], wgu_s [E][2I/128][D/128]: gate and up interleaved by

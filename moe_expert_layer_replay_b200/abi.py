@@ -23,7 +23,7 @@ EXPORTS = [
     "moe_combine_bwd", "moe_unpermute_reduce", "moe_permute_noalloc", "moe_kernel_launches",
     "moe_router_fwd", "moe_capture_payload", "moe_router_bwd_workspace_size", "moe_router_bwd",
     "moe_grouped_gemm_fp8_seg", "moe_gateup_gather_fp8", "moe_set_gemm_variant", "moe_quant_nvfp4",
-    "moe_gemm_pair_clusters",
+    "moe_gemm_pair_clusters", "moe_gemm_nvfp4",
 ]
 
 
@@ -79,7 +79,8 @@ def lib() -> ctypes.CDLL:
             "moe_permute_noalloc": (ctypes.c_int, [P, D, P, P, P, P, P, P, P, P]),
             "moe_quant_fp8_block": (ctypes.c_int, [P, I64, I64, I64, I32, I32, P, P, P, P, P]),
             "moe_quant_weights": (ctypes.c_int, [P, P, P, D, P, P, P, P, P, P, P, P, P]),
-            "moe_quant_nvfp4": (ctypes.c_int, [P, I64, I64, I64, P, P, P, P, P]),
+            "moe_quant_nvfp4": (ctypes.c_int, [P, I64, I64, I64, P, P, I32, P, P, P]),
+            "moe_gemm_nvfp4": (ctypes.c_int, [I64, I32, I32, I32, P, P, P, P, P, P, P, P, P]),
             "moe_grouped_gemm_fp8": (ctypes.c_int, [I32, D, P, ctypes.POINTER(GemmArgs), P]),
             "moe_grouped_gemm_fp8_seg": (ctypes.c_int, [I32, D, I64, P, I32, ctypes.POINTER(GemmArgs), P]),
             "moe_gateup_gather_fp8": (ctypes.c_int, [D, P, P, ctypes.POINTER(GemmArgs), P]),
@@ -202,11 +203,21 @@ def quant_fp8_block(inp, rows, cols, ld, blk_r, blk_c, q, s, qT=None, sT=None, s
                                                             int(blk_c), _p(q), _p(s), _p(qT), _p(sT), _s(stream)))
 
 
-def quant_nvfp4(inp, rows, cols, ld, q, sf, amax, s_g, stream=None):
-    """NVFP4: packed e2m1 codes q [rows, cols/2], e4m3 block scales sf [rows, cols/16],
-    tensor amax and scale s_g (one float each, device)."""
-    _check("moe_quant_nvfp4", lib().moe_quant_nvfp4(_p(inp), int(rows), int(cols), int(ld), _p(q), _p(sf), _p(amax),
-                                                    _p(s_g), _s(stream)))
+NVFP4_SF_ROWS, NVFP4_SF_MMA = 0, 1
+
+
+def quant_nvfp4(inp, rows, cols, ld, q, sf, amax, s_g, sf_layout=NVFP4_SF_ROWS, stream=None):
+    """NVFP4: packed e2m1 codes q [rows, cols/2], e4m3 block scales sf ([rows, cols/16], or the
+    block-scaled MMA's atoms with NVFP4_SF_MMA), tensor amax and scale s_g (one float each, device)."""
+    _check("moe_quant_nvfp4", lib().moe_quant_nvfp4(_p(inp), int(rows), int(cols), int(ld), _p(q), _p(sf),
+                                                    int(sf_layout), _p(amax), _p(s_g), _s(stream)))
+
+
+def gemm_nvfp4(rows_cap, N, K, n_seg, offsets, a, sfa, a_sg, b, sfb, b_sg, out, stream=None):
+    """NVFP4 grouped GEMM: out [rows_cap, N] fp32 = value(A) value(B_e)^T per segment."""
+    _check("moe_gemm_nvfp4", lib().moe_gemm_nvfp4(int(rows_cap), int(N), int(K), int(n_seg), _p(offsets), _p(a),
+                                                  _p(sfa), _p(a_sg), _p(b), _p(sfb), _p(b_sg), _p(out),
+                                                  _s(stream)))
 
 
 def quant_weights(w_gate, w_up, w_down, d: Dims, wgu_q, wgu_s, wd_q, wd_s,

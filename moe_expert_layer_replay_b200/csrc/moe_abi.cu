@@ -244,14 +244,34 @@ int moe_quant_fp8_block(const uint16_t *in, int64_t rows, int64_t cols, int64_t 
 }
 
 int moe_quant_nvfp4(const uint16_t *in, int64_t rows, int64_t cols, int64_t ld, uint8_t *q, uint8_t *sf,
-                    float *amax, float *s_g, void *stream)
+                    int32_t sf_layout, float *amax, float *s_g, void *stream)
 {
     if (rows < 0 || cols <= 0 || cols % 16 || ld < cols || ld % 8) return MOE_ERR_INVALID_ARG;
+    if (sf_layout != MOE_NVFP4_SF_ROWS && sf_layout != MOE_NVFP4_SF_MMA) return MOE_ERR_INVALID_ARG;
+    if (sf_layout == MOE_NVFP4_SF_MMA && (rows % 128 || cols % 64)) return MOE_ERR_INVALID_ARG;
     if (!amax || !s_g || !aligned4(amax) || !aligned4(s_g)) return MOE_ERR_INVALID_ARG;
     if (rows > 0 && (!in || !q || !sf || !aligned16(in) || !aligned8(q))) return MOE_ERR_INVALID_ARG;
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    return moe::launch_quant_nvfp4(in, rows, cols, ld, q, sf, amax, s_g, sms, as_stream(stream));
+    return moe::launch_quant_nvfp4(in, rows, cols, ld, q, sf, sf_layout == MOE_NVFP4_SF_MMA, amax, s_g, sms,
+                                   as_stream(stream));
+}
+
+int moe_gemm_nvfp4(int64_t rows_cap, int32_t N, int32_t K, int32_t n_seg, const int32_t *offsets,
+                   const uint8_t *a, const uint8_t *sfa, const float *a_sg, const uint8_t *b, const uint8_t *sfb,
+                   const float *b_sg, float *out, void *stream)
+{
+    if (rows_cap < 0 || rows_cap % 128 || N <= 0 || N % 256 || K <= 0 || K % 256 || n_seg <= 0 || n_seg > 256)
+        return MOE_ERR_INVALID_ARG;
+    if (!offsets || !a || !sfa || !a_sg || !b || !sfb || !b_sg || !out) return MOE_ERR_INVALID_ARG;
+    for (const void *p : {(const void *)a, (const void *)sfa, (const void *)b, (const void *)sfb, (const void *)out})
+        if (!aligned16(p)) return MOE_ERR_INVALID_ARG;
+    if (!aligned4(a_sg) || !aligned4(b_sg)) return MOE_ERR_INVALID_ARG;
+    if (rows_cap == 0) return MOE_OK;
+    int *sp = status_ptr();
+    if (!sp) return MOE_ERR_CUDA;
+    return moe::launch_gemm_nvfp4(rows_cap, N, K, n_seg, offsets, a, sfa, a_sg, b, sfb, b_sg, out, sp,
+                                  wait_budget(), as_stream(stream));
 }
 
 int moe_quant_weights(const uint16_t *w_gate, const uint16_t *w_up, const uint16_t *w_down,

@@ -65,9 +65,18 @@ __global__ void __launch_bounds__(256) amax_kernel(const uint16_t *__restrict__ 
     }
 }
 
+// Byte of the scale of (row r, 16-element group b) in the MMA's layout: 512-byte
+// atoms per (128-row block, 64-element K step), K steps of a row block
+// consecutive; inside an atom, row 32 r1 + r0, group j at byte 16 r0 + 4 r1 + j.
+__device__ __forceinline__ int64_t sf_mma_offset(int64_t r, int64_t b, int64_t cols)
+{
+    const int64_t rb = r >> 7, rr = r & 127, ks = b >> 2, j = b & 3;
+    return ((rb * (cols / 64) + ks) << 9) + ((rr & 31) << 4) + ((rr >> 5) << 2) + j;
+}
+
 __global__ void __launch_bounds__(256) quant_kernel(const uint16_t *__restrict__ in, int64_t rows, int64_t cols,
                                                     int64_t ld, const float *__restrict__ amax,
-                                                    uint8_t *__restrict__ q, uint8_t *__restrict__ sf,
+                                                    uint8_t *__restrict__ q, uint8_t *__restrict__ sf, bool sf_mma,
                                                     float *__restrict__ s_g_out)
 {
     const float s_g = tensor_scale(*amax);
@@ -91,13 +100,13 @@ __global__ void __launch_bounds__(256) quant_kernel(const uint16_t *__restrict__
         out = make_uint2(e2m1x8(v), e2m1x8(v + 8));
     }
     *reinterpret_cast<uint2 *>(q + r * (cols / 2) + 8 * b) = out;
-    sf[r * nb + b] = (uint8_t)code;
+    sf[sf_mma ? sf_mma_offset(r, b, cols) : r * nb + b] = (uint8_t)code;
 }
 
 }  // namespace nvfp4
 
 int launch_quant_nvfp4(const uint16_t *in, int64_t rows, int64_t cols, int64_t ld, uint8_t *q, uint8_t *sf,
-                       float *amax, float *s_g, int sms, cudaStream_t s)
+                       bool sf_mma, float *amax, float *s_g, int sms, cudaStream_t s)
 {
     if (cudaMemsetAsync(amax, 0, sizeof(float), s) != cudaSuccess) return MOE_ERR_CUDA;
     if (rows > 0) {
@@ -109,7 +118,7 @@ int launch_quant_nvfp4(const uint16_t *in, int64_t rows, int64_t cols, int64_t l
     }
     const int64_t blocks = rows * (cols / 16);
     nvfp4::quant_kernel<<<(unsigned)((blocks + 255) / 256 > 0 ? (blocks + 255) / 256 : 1), 256, 0, s>>>(
-        in, rows, cols, ld, amax, q, sf, s_g);
+        in, rows, cols, ld, amax, q, sf, sf_mma, s_g);
     count_launch();
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -6,7 +6,7 @@ import numpy as np
 import pytest
 import torch
 
-from _util import dev, host, same_bits
+from _util import close, dev, host, same_bits
 
 pytestmark = pytest.mark.gpu
 
@@ -52,3 +52,93 @@ def test_quant_nvfp4_matches_oracle(A, orc, name):
     same_bits(host(s_g), np.array([sg], np.float32), "tensor scale")
     same_bits(host(sf), S8, "e4m3 block scales")
     same_bits(host(q), nvfp4.pack(codes), "packed e2m1 codes")
+
+
+def sf_mma_layout(S8):
+    """[rows][cols/16] e4m3 scale codes -> the block-scaled MMA's atom layout
+    (512-byte atoms per 128-row block and 64-column step, K steps of a row
+    block consecutive; row 32 r1 + r0, group j of a step at byte 16 r0 + 4 r1
+    + j), as moe.h states it."""
+    rows, nb = S8.shape
+    r = np.arange(rows)[:, None]
+    b = np.arange(nb)[None, :]
+    rr = r & 127
+    off = ((r >> 7) * (nb // 4) + (b >> 2)) * 512 + (rr & 31) * 16 + (rr >> 5) * 4 + (b & 3)
+    out = np.zeros(rows * nb, np.uint8)
+    out[off.ravel()] = S8.ravel()
+    return out
+
+
+def test_quant_nvfp4_mma_layout(A, orc):
+    from oracle import nvfp4
+    from moe_expert_layer_replay_b200.inputs import to_bf16_bits
+    rng = np.random.default_rng(96)
+    x = to_bf16_bits((rng.standard_normal((384, 1024)) * np.exp(rng.uniform(-4, 4, (384, 1)))).astype(np.float32))
+    q = torch.empty(384, 512, dtype=torch.uint8, device="cuda")
+    sf = torch.full((384 * 64,), 0xAA, dtype=torch.uint8, device="cuda")
+    amax = torch.empty(1, device="cuda")
+    s_g = torch.empty(1, device="cuda")
+    A.quant_nvfp4(dev(x), 384, 1024, 1024, q, sf, amax, s_g, sf_layout=A.NVFP4_SF_MMA)
+    torch.cuda.synchronize()
+    codes, S8, sg = nvfp4.quant(x)
+    same_bits(host(sf), sf_mma_layout(S8), "e4m3 block scales, MMA layout")
+    same_bits(host(q), nvfp4.pack(codes), "packed e2m1 codes")
+    same_bits(host(s_g), np.array([sg], np.float32), "tensor scale")
+    with pytest.raises(A.MoeError):   # the MMA layout needs whole 128-row blocks
+        A.quant_nvfp4(dev(x[:200]), 200, 1024, 1024, q, sf, amax, s_g, sf_layout=A.NVFP4_SF_MMA)
+
+
+# segment row counts (multiples of 128, 0 = an empty segment), N, K
+GEMM_CASES = {
+    "one_tile": ([128], 256, 256),
+    "grouped_empty_segment": ([128, 0, 384], 512, 768),
+    "ffn_shape": ([256, 512, 128, 384], 2048, 2048),
+    "deep_k": ([256], 256, 7168),
+}
+
+
+@pytest.mark.parametrize("case", list(GEMM_CASES))
+def test_gemm_nvfp4_matches_oracle(A, orc, case):
+    """The NVFP4 grouped GEMM against the oracle's fp64 product of the
+    dequantised operands (oracle.nvfp4.gemm), per segment.  Both sides use the
+    same codes and scales (the GPU quantiser's, equal to the oracle's bit for
+    bit by the tests above); each product of two NVFP4 values is exact in fp32
+    (at most 12 significant bits), so the kernel differs from the oracle only
+    by its fp32 accumulation order and the final scaling: a relative error of
+    order 1e-7, checked at 1e-5 (Frobenius) and 1e-4 * rms (max-abs)."""
+    from oracle import nvfp4
+    counts, N, K = GEMM_CASES[case]
+    E = len(counts)
+    rng = np.random.default_rng(97 + N + K)
+    offs = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    R = int(offs[-1]) + 128   # one spare row block past the last segment
+    from moe_expert_layer_replay_b200.inputs import to_bf16_bits
+    x = to_bf16_bits(rng.standard_normal((R, K)).astype(np.float32))
+    x[offs[-1]:] = 0
+    W = to_bf16_bits((rng.standard_normal((E, N, K)) * 0.02).astype(np.float32))
+    aq = torch.empty(R, K // 2, dtype=torch.uint8, device="cuda")
+    asf = torch.empty(R * K // 16, dtype=torch.uint8, device="cuda")
+    amax = torch.empty(1, device="cuda")
+    a_sg = torch.empty(1, device="cuda")
+    A.quant_nvfp4(dev(x), R, K, K, aq, asf, amax, a_sg, sf_layout=A.NVFP4_SF_MMA)
+    bq = torch.empty(E, N, K // 2, dtype=torch.uint8, device="cuda")
+    bsf = torch.empty(E, N * K // 16, dtype=torch.uint8, device="cuda")
+    bamax = torch.empty(E, device="cuda")
+    b_sg = torch.empty(E, device="cuda")
+    Wd = dev(W)
+    for e in range(E):
+        A.quant_nvfp4(Wd[e], N, K, K, bq[e], bsf[e], bamax[e:e + 1], b_sg[e:e + 1], sf_layout=A.NVFP4_SF_MMA)
+    out = torch.full((R, N), -7.0, dtype=torch.float32, device="cuda")
+    A.gemm_nvfp4(R, N, K, E, dev(offs), aq, asf, a_sg, bq, bsf, b_sg, out)
+    torch.cuda.synchronize()
+    assert A.get_status() == A.OK
+    got = host(out)
+    ca, Sa, sga = nvfp4.quant(x)
+    for e in range(E):
+        r0, r1 = int(offs[e]), int(offs[e + 1])
+        if r1 == r0:
+            continue
+        cb, Sb, sgb = nvfp4.quant(W[e])
+        ref = nvfp4.gemm(ca[r0:r1], Sa[r0:r1], sga, cb, Sb, sgb)
+        close(got[r0:r1], ref, rel_fro=1e-5, max_abs_rms=1e-4, what=f"{case}: segment {e}")
+    assert np.all(got[offs[-1]:] == -7.0), "rows past the last segment are untouched"
