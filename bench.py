@@ -613,21 +613,21 @@ def nvfp4_stages(abi, d, B, x, wg, wu, R_pad):
     rows[ok] = x[src[ok] // d.k]
     wgu = torch.cat([wg, wu], dim=1).contiguous()          # [E][2I][D]
     q = torch.empty(R_cap, D // 2, dtype=torch.uint8, device="cuda")
-    sf = torch.empty(R_cap * D // 16, dtype=torch.uint8, device="cuda")
+    sf = torch.empty(4 * R_cap * D // 16, dtype=torch.uint8, device="cuda")
     amax = torch.empty(1, device="cuda")
     sg = torch.empty(1, device="cuda")
     wq = torch.empty(E, 2 * I, D // 2, dtype=torch.uint8, device="cuda")
-    wsf = torch.empty(E, 2 * I * D // 16, dtype=torch.uint8, device="cuda")
+    wsf = torch.empty(E, 4 * 2 * I * D // 16, dtype=torch.uint8, device="cuda")
     wamax = torch.empty(E, device="cuda")
     wsg = torch.empty(E, device="cuda")
     for e in range(E):
         abi.quant_nvfp4(wgu[e], 2 * I, D, D, wq[e], wsf[e], wamax[e:e + 1], wsg[e:e + 1],
-                        sf_layout=abi.NVFP4_SF_MMA)
+                        sf_layout=abi.NVFP4_SF_MMA_B)
     out = torch.empty(R_cap, 2 * I, dtype=torch.float32, device="cuda")
     return [
         ("NVFP4 quant of the permuted rows", lambda: abi.quant_nvfp4(rows, R_cap, D, D, q, sf, amax, sg,
-                                                                      sf_layout=abi.NVFP4_SF_MMA),
-         "B", 2 * 2 * R_cap * D + R_cap * (D // 2 + D // 16)),
+                                                                      sf_layout=abi.NVFP4_SF_MMA_A),
+         "B", 2 * 2 * R_cap * D + R_cap * (D // 2 + 4 * D // 16)),
         ("gemm gate/up NVFP4 (fp32 out)", lambda: abi.gemm_nvfp4(R_cap, 2 * I, D, E, B.offsets, q, sf, sg, wq, wsf,
                                                                   wsg, out),
          "F4", 4.0 * d.T * d.k * D * I),

@@ -232,13 +232,21 @@ int moe_quant_fp8_block(const uint16_t *in, int64_t rows, int64_t cols, int64_t 
  *   sf                e4m3 block-scale codes e4m3(RNE, satfinite)(
  *                     fp32(fp32(amax_b / 6) * s_g)), amax_b over 16 elements,
  *                     laid out by sf_layout:
- *                       MOE_NVFP4_SF_ROWS  [rows][cols/16];
- *                       MOE_NVFP4_SF_MMA   the block-scaled MMA's layout
- *                         (rows % 128 == 0, cols % 64 == 0): 512-byte atoms,
- *                         atom (rb, ks) of 128-row block rb and 64-column step
- *                         ks at (rb * cols/64 + ks) * 512; inside it the scale
- *                         of row 128 rb + 32 r1 + r0, group 4 ks + j at byte
- *                         16 r0 + 4 r1 + j;
+ *                       MOE_NVFP4_SF_ROWS   [rows][cols/16];
+ *                       MOE_NVFP4_SF_MMA_A  the NVFP4 GEMM's A-side layout
+ *                         (rows % 128 == 0, cols % 128 == 0), 4 * rows * cols/16 bytes;
+ *                       MOE_NVFP4_SF_MMA_B  its B-side layout (rows % 256 == 0,
+ *                         cols % 64 == 0), 4 * rows * cols/16 bytes.
+ *                     Both store every scale four times, the image that
+ *                     tcgen05.cp 128x256b copies into TMEM lanes 0-127: a
+ *                     4096-byte block holds, for lane l and half h, the scales
+ *                     of rows 32 r1 + l % 32 (r1 = 0..3) of one 128-row block for
+ *                     one 64-column step (row 32 r1 + l % 32, group j at byte
+ *                     4 r1 + j of the 16) at (l >> 3) * 256 + h * 128 + (l & 7) * 16.
+ *                     A: block (row block rb, step pair kp) at (rb * cols/128 + kp)
+ *                     * 4096, h = step 2 kp + h.  B: block (row-block pair rbp,
+ *                     step ks) at (rbp * cols/64 + ks) * 4096, h = row block
+ *                     2 rbp + h;
  *   q  [rows][cols/2] e2m1 codes, two per byte (element 2i in the low
  *                     nibble): 0 where the block scale is 0, else e2m1(RNE,
  *                     satfinite)(fp32(x * fp32(s_g / value(sf)))).
@@ -246,7 +254,8 @@ int moe_quant_fp8_block(const uint16_t *in, int64_t rows, int64_t cols, int64_t 
  * words the call writes (amax is zeroed first, then accumulated).
  * MOE_ERR_INVALID_ARG for an unknown layout or shapes the layout excludes. */
 #define MOE_NVFP4_SF_ROWS 0
-#define MOE_NVFP4_SF_MMA 1
+#define MOE_NVFP4_SF_MMA_A 1
+#define MOE_NVFP4_SF_MMA_B 2
 int moe_quant_nvfp4(const uint16_t *in, int64_t rows, int64_t cols, int64_t ld, uint8_t *q, uint8_t *sf,
                     int32_t sf_layout, float *amax, float *s_g, void *stream);
 
@@ -255,10 +264,11 @@ int moe_quant_nvfp4(const uint16_t *in, int64_t rows, int64_t cols, int64_t ld, 
  *   out[r][n] = sum_k value(A)[r][k] * value(B_e)[n][k]   for r in segment e,
  * segments [offsets[e], offsets[e+1]) of the rows, 128-aligned (n_seg <= 256;
  * offsets on the device, read there).  Operands as moe_quant_nvfp4 makes
- * them with MOE_NVFP4_SF_MMA:
- *   a    [rows_cap][K/2] packed e2m1 codes;   sfa  scale atoms of A (rows_cap rows);
+ * them:
+ *   a    [rows_cap][K/2] packed e2m1 codes;  sfa  A's scales, MOE_NVFP4_SF_MMA_A;
  *   a_sg A's tensor scale (device float);
- *   b    [n_seg][N][K/2] codes of each segment's B;  sfb  their atoms (n_seg * N rows);
+ *   b    [n_seg][N][K/2] codes of each segment's B;  sfb  their scales,
+ *        MOE_NVFP4_SF_MMA_B over the n_seg * N rows;
  *   b_sg [n_seg] tensor scales of the B's (device);
  *   out  [rows_cap][N] fp32, rows past offsets[n_seg] untouched.
  * N % 256 == 0, K % 256 == 0, rows_cap % 128 == 0; pointers 16-byte aligned

@@ -203,12 +203,13 @@ def quant_fp8_block(inp, rows, cols, ld, blk_r, blk_c, q, s, qT=None, sT=None, s
                                                             int(blk_c), _p(q), _p(s), _p(qT), _p(sT), _s(stream)))
 
 
-NVFP4_SF_ROWS, NVFP4_SF_MMA = 0, 1
+NVFP4_SF_ROWS, NVFP4_SF_MMA_A, NVFP4_SF_MMA_B = 0, 1, 2
 
 
 def quant_nvfp4(inp, rows, cols, ld, q, sf, amax, s_g, sf_layout=NVFP4_SF_ROWS, stream=None):
     """NVFP4: packed e2m1 codes q [rows, cols/2], e4m3 block scales sf ([rows, cols/16], or the
-    block-scaled MMA's atoms with NVFP4_SF_MMA), tensor amax and scale s_g (one float each, device)."""
+    NVFP4 GEMM's A- or B-side layout: NVFP4_SF_MMA_A / _B, 4 * rows * cols/16 bytes), tensor amax
+    and scale s_g (one float each, device)."""
     _check("moe_quant_nvfp4", lib().moe_quant_nvfp4(_p(inp), int(rows), int(cols), int(ld), _p(q), _p(sf),
                                                     int(sf_layout), _p(amax), _p(s_g), _s(stream)))
 

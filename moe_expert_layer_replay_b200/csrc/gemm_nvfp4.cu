@@ -15,23 +15,25 @@
 // Design (one persistent CTA per SM, 12 warps):
 //   warp 0     TMA producer: per 256-element K block, A (128 rows x 128 B),
 //              B (256 rows x 128 B), both 128-byte swizzled, and the scale
-//              factors of both (bulk copies of their 512-byte atoms) into a
-//              4-stage ring;
+//              factors of both (one bulk copy each) into a 3-stage ring;
 //   warp 1     allocates 512 TMEM columns; lane 0 copies each K block's
-//              scale factors from shared memory into TMEM (tcgen05.cp
-//              32x128b.warpx4) and issues four MMAs (M=128, N=256, K=64);
+//              scale factors from shared memory into TMEM (six tcgen05.cp
+//              128x256b) and issues four MMAs (M=128, N=256, K=64);
 //   warps 4-11 epilogue (TMEM lane quarter warp % 4, column half (warp - 4) / 4).
 // TMEM: the accumulator in columns 0-255; scale-factor slot s (one per ring
 // stage) in columns 256 + 48 s: A's four K steps (4 columns each), then B's
 // (8 columns each: rows 0-127, then rows 128-255).
 //
-// Scale-factor layout (global and shared): for a matrix of R rows (R % 128
-// == 0) and K elements (K % 64 == 0), the atom of row block rb and K step ks
-// (64 elements) is 512 bytes at (rb * K/64 + ks) * 512; inside it, the scale
-// of row 32 r1 + r0 for the 16-element group j is at byte 16 r0 + 4 r1 + j.
-// tcgen05.cp 32x128b.warpx4 gives TMEM lane 32 q + r0 (every q) the 16 bytes
-// of line r0, so row m's scales sit in column m / 32 of the atom's four,
-// byte j: the layout the MMA reads.
+// Scale layout the MMA reads (one K step, one 128-row block): TMEM lane
+// 32 q + r0 (every q), four columns, column r1 byte j = the scale of row
+// 32 r1 + r0, group j.  The global and shared images (moe.h, MOE_NVFP4_SF_MMA_A
+// / _B) hold those lanes' bytes already replicated, as 4096-byte blocks of two
+// such atoms that one tcgen05.cp 128x256b moves into 8 columns: for A a pair
+// of K steps (SFA of step ks at 4 ks), for B the two 128-row blocks of one K
+// step (SFB of step ks at 8 ks).  A copy instruction costs about 60 cycles of
+// the MMA thread whatever its size (measured: twelve 32x128b.warpx4 copies of
+// the compact atoms took 720 cycles per K block, six 128x256b 340), so the
+// fourfold replication in memory buys half the copies.
 //
 // Every mbarrier wait is bounded; on expiry the kernel latches
 // MOE_ERR_TIMEOUT, drains what it issued, frees TMEM and returns.
@@ -46,15 +48,15 @@ using namespace sm100;
 constexpr int BM = 128, BN = 256;
 constexpr int KB_ELEMS = 256;   // e2m1 elements of K per stage (128 bytes per row)
 constexpr int KB_BYTES = KB_ELEMS / 2;
-constexpr int STAGES = 4;
+constexpr int STAGES = 3;
 constexpr int NUM_THREADS = 384;
 constexpr int EPI_WARP0 = 4;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int A_BYTES = BM * KB_BYTES;        // 16 KB
 constexpr int B_BYTES = BN * KB_BYTES;        // 32 KB
-constexpr int ATOM = 512;
-constexpr int SFA_BYTES = 4 * ATOM;           // four K steps, one 128-row atom each
-constexpr int SFB_BYTES = 8 * ATOM;           // four K steps, two 128-row atoms each
+constexpr int SF_BLOCK = 4096;                // one tcgen05.cp 128x256b source (two atoms, x4 lanes)
+constexpr int SFA_BYTES = 2 * SF_BLOCK;       // two K-step pairs
+constexpr int SFB_BYTES = 4 * SF_BLOCK;       // four K steps, both row blocks
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
 constexpr int OFF_BAR = STAGES * STAGE_BYTES;
 constexpr int OFF_TMEM_SLOT = OFF_BAR + (2 * STAGES + 3) * 8;
@@ -83,30 +85,31 @@ __device__ __forceinline__ void mma_nvf4(uint32_t d, uint64_t a, uint64_t b, uin
         "l"(a), "l"(b), "r"(IDESC), "r"(sfa), "r"(sfb), "r"(accum));
 }
 
-// Shared-memory descriptor of one 512-byte scale-factor atom for tcgen05.cp:
-// K-major, no swizzle, 8-row core matrices of 16-byte rows, consecutive
-// (stride byte offset 128; a single core matrix along K).
+// Shared-memory descriptor of one 4096-byte scale block for tcgen05.cp
+// 128x256b: K-major, no swizzle, 8-row core matrices of 16-byte rows; the two
+// 16-byte halves of a lane's 32 bytes 128 bytes apart (leading byte offset),
+// row groups 256 bytes apart (stride byte offset).
 __device__ __forceinline__ uint64_t sf_desc(uint32_t saddr)
 {
     uint64_t d = 0;
     d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
-    d |= (uint64_t)(128 >> 4) << 16;   // leading byte offset (one core matrix along K)
-    d |= (uint64_t)(128 >> 4) << 32;   // stride byte offset
+    d |= (uint64_t)(128 >> 4) << 16;   // leading byte offset
+    d |= (uint64_t)(256 >> 4) << 32;   // stride byte offset
     d |= (uint64_t)1 << 46;            // descriptor version
     return d;                          // layout type 0: no swizzle
 }
 
 __device__ __forceinline__ void sf_copy(uint32_t taddr, uint64_t desc)
 {
-    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc) : "memory");
+    asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(desc) : "memory");
 }
 
 struct Args {
     const int32_t *offsets;   // [n_seg + 1], 128-aligned
     int n_seg;
     int N, K;                 // output columns (% 256 == 0), reduction length (% 256 == 0)
-    const uint8_t *sfa;       // A scale atoms [R_cap/128][K/64][512]
-    const uint8_t *sfb;       // B scale atoms [n_seg*N/128][K/64][512]
+    const uint8_t *sfa;       // A scales, blocks [R_cap/128][K/128][4096]
+    const uint8_t *sfb;       // B scales, blocks [n_seg*N/256][K/64][4096]
     const float *a_sg;        // A's tensor scale (one float)
     const float *b_sg;        // each segment's B tensor scale [n_seg]
     float *out;               // [R_cap][N]
@@ -184,9 +187,8 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
             for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
                 const Tile x = tile_of(t, p, offs_s);
                 const int brow = x.e * p.N + x.n0;
-                const uint8_t *sfa = p.sfa + ((int64_t)(x.m0 / 128) * KS) * ATOM;
-                const uint8_t *sfb0 = p.sfb + ((int64_t)(brow / 128) * KS) * ATOM;
-                const uint8_t *sfb1 = sfb0 + (int64_t)KS * ATOM;
+                const uint8_t *sfa = p.sfa + ((int64_t)(x.m0 / 128) * (KS / 2)) * SF_BLOCK;
+                const uint8_t *sfb = p.sfb + ((int64_t)(brow / 256) * KS) * SF_BLOCK;
                 for (int kb = 0; kb < KB; ++kb) {
                     if (!wait_bounded(bar_empty + 8 * stage, phase ^ 1, p.budget, abort_flag, p.status)) {
                         ok = false;
@@ -199,9 +201,8 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
                     mbar_arrive_expect_tx(fb, STAGE_BYTES);
                     tma_load_2d(dA, &tmA, kb * KB_BYTES, x.m0, fb);
                     tma_load_2d(dB, &tmB, kb * KB_BYTES, brow, fb);
-                    bulk_g2s(dSA, sfa + (int64_t)4 * kb * ATOM, SFA_BYTES, fb);
-                    bulk_g2s(dSB, sfb0 + (int64_t)4 * kb * ATOM, 4 * ATOM, fb);
-                    bulk_g2s(dSB + 4 * ATOM, sfb1 + (int64_t)4 * kb * ATOM, 4 * ATOM, fb);
+                    bulk_g2s(dSA, sfa + (int64_t)2 * kb * SF_BLOCK, SFA_BYTES, fb);
+                    bulk_g2s(dSB, sfb + (int64_t)4 * kb * SF_BLOCK, SFB_BYTES, fb);
                     pend |= 1u << stage;
                     pend_phase = (pend_phase & ~(1u << stage)) | (phase << stage);
                     if (++stage == STAGES) {
@@ -237,12 +238,10 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
                     const uint32_t dA = sbase + stage * STAGE_BYTES, dB = dA + A_BYTES;
                     const uint32_t dSA = dB + B_BYTES, dSB = dSA + SFA_BYTES;
                     const uint32_t sf = tmem_base + SF_COL0 + SF_SLOT_COLS * (uint32_t)stage;
+                    sf_copy(sf, sf_desc(dSA));
+                    sf_copy(sf + 8, sf_desc(dSA + SF_BLOCK));
 #pragma unroll
-                    for (int ks = 0; ks < 4; ++ks) {
-                        sf_copy(sf + 4 * ks, sf_desc(dSA + ks * ATOM));
-                        sf_copy(sf + 16 + 8 * ks, sf_desc(dSB + ks * ATOM));
-                        sf_copy(sf + 16 + 8 * ks + 4, sf_desc(dSB + 4 * ATOM + ks * ATOM));
-                    }
+                    for (int ks = 0; ks < 4; ++ks) sf_copy(sf + 16 + 8 * ks, sf_desc(dSB + ks * SF_BLOCK));
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks)
                         mma_nvf4(tmem_base, sdesc(dA + 32 * ks), sdesc(dB + 32 * ks), sf + 4 * ks, sf + 16 + 8 * ks,
@@ -275,26 +274,25 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
             tc_fence_after();
             const float inv = __fdiv_rn(1.0f, a_sg * p.b_sg[x.e]);
             float *o = p.out + ((int64_t)x.m0 + row) * p.N + x.n0 + 128 * h;
-#pragma unroll 1
-            for (int g = 0; g < 2; ++g) {   // 64 columns per wait
-                uint32_t r[64];
+            // the warp's 128 columns read at once, the accumulator handed back to
+            // the next tile's MMAs, then scaled and stored (the stores no longer
+            // hold the tensor core: measured, 6.7k cycles per tile with reads and
+            // stores interleaved)
+            uint32_t r[128];
 #pragma unroll
-                for (int j = 0; j < 4; ++j) MOE_TMEM_LD16(lane_addr + (uint32_t)(64 * g + 16 * j), (r + 16 * j));
-                tmem_wait_ld();
-                if (g == 1) {   // the accumulator has been read: the next tile's MMAs may start
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(bar_tempty);
-                }
+            for (int j = 0; j < 8; ++j) MOE_TMEM_LD16(lane_addr + (uint32_t)(16 * j), (r + 16 * j));
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_tempty);
 #pragma unroll
-                for (int i = 0; i < 64; i += 4) {
-                    float4 v;
-                    v.x = __uint_as_float(r[i]) * inv;
-                    v.y = __uint_as_float(r[i + 1]) * inv;
-                    v.z = __uint_as_float(r[i + 2]) * inv;
-                    v.w = __uint_as_float(r[i + 3]) * inv;
-                    *reinterpret_cast<float4 *>(o + 64 * g + i) = v;
-                }
+            for (int i = 0; i < 128; i += 4) {
+                float4 v;
+                v.x = __uint_as_float(r[i]) * inv;
+                v.y = __uint_as_float(r[i + 1]) * inv;
+                v.z = __uint_as_float(r[i + 2]) * inv;
+                v.w = __uint_as_float(r[i + 3]) * inv;
+                *reinterpret_cast<float4 *>(o + i) = v;
             }
         }
     }

@@ -39,7 +39,7 @@ int launch_capture(const int32_t *idx, int T, int k, int layer, int32_t *payload
 int launch_router_bwd(const float *dz, const uint16_t *x, const uint16_t *w_r, int T, int D, int E,
                       const uint16_t *dx_in, uint16_t *dx, float *dw_r, void *ws, cudaStream_t s);
 int launch_quant_nvfp4(const uint16_t *in, int64_t rows, int64_t cols, int64_t ld, uint8_t *q, uint8_t *sf,
-                       bool sf_mma, float *amax, float *s_g, int sms, cudaStream_t s);
+                       int sf_layout, float *amax, float *s_g, int sms, cudaStream_t s);
 int launch_gemm_nvfp4(int64_t R_cap, int N, int K, int n_seg, const int32_t *offsets, const uint8_t *a,
                       const uint8_t *sfa, const float *a_sg, const uint8_t *b, const uint8_t *sfb,
                       const float *b_sg, float *out, int *status, uint64_t budget, cudaStream_t s);

@@ -247,14 +247,15 @@ int moe_quant_nvfp4(const uint16_t *in, int64_t rows, int64_t cols, int64_t ld, 
                     int32_t sf_layout, float *amax, float *s_g, void *stream)
 {
     if (rows < 0 || cols <= 0 || cols % 16 || ld < cols || ld % 8) return MOE_ERR_INVALID_ARG;
-    if (sf_layout != MOE_NVFP4_SF_ROWS && sf_layout != MOE_NVFP4_SF_MMA) return MOE_ERR_INVALID_ARG;
-    if (sf_layout == MOE_NVFP4_SF_MMA && (rows % 128 || cols % 64)) return MOE_ERR_INVALID_ARG;
+    if (sf_layout != MOE_NVFP4_SF_ROWS && sf_layout != MOE_NVFP4_SF_MMA_A && sf_layout != MOE_NVFP4_SF_MMA_B)
+        return MOE_ERR_INVALID_ARG;
+    if (sf_layout == MOE_NVFP4_SF_MMA_A && (rows % 128 || cols % 128)) return MOE_ERR_INVALID_ARG;
+    if (sf_layout == MOE_NVFP4_SF_MMA_B && (rows % 256 || cols % 64)) return MOE_ERR_INVALID_ARG;
     if (!amax || !s_g || !aligned4(amax) || !aligned4(s_g)) return MOE_ERR_INVALID_ARG;
     if (rows > 0 && (!in || !q || !sf || !aligned16(in) || !aligned8(q))) return MOE_ERR_INVALID_ARG;
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    return moe::launch_quant_nvfp4(in, rows, cols, ld, q, sf, sf_layout == MOE_NVFP4_SF_MMA, amax, s_g, sms,
-                                   as_stream(stream));
+    return moe::launch_quant_nvfp4(in, rows, cols, ld, q, sf, sf_layout, amax, s_g, sms, as_stream(stream));
 }
 
 int moe_gemm_nvfp4(int64_t rows_cap, int32_t N, int32_t K, int32_t n_seg, const int32_t *offsets,

@@ -65,18 +65,29 @@ __global__ void __launch_bounds__(256) amax_kernel(const uint16_t *__restrict__ 
     }
 }
 
-// Byte of the scale of (row r, 16-element group b) in the MMA's layout: 512-byte
-// atoms per (128-row block, 64-element K step), K steps of a row block
-// consecutive; inside an atom, row 32 r1 + r0, group j at byte 16 r0 + 4 r1 + j.
-__device__ __forceinline__ int64_t sf_mma_offset(int64_t r, int64_t b, int64_t cols)
+// The block-scaled MMA's scale layouts (as tcgen05.cp 128x256b copies them
+// into TMEM, four copies of every scale, one per TMEM lane quarter).  A 4096-
+// byte block holds, for TMEM lane l (0..127) and half h, the 16 bytes of
+// "line" l % 32 of one 128-row, 64-element atom (row 32 r1 + l % 32, group j
+// at byte 4 r1 + j), at (l >> 3) * 256 + h * 128 + (l & 7) * 16: 8-row core
+// matrices, the two halves 128 bytes apart, row groups 256 bytes apart.
+//   A side: block (row block rb, K-step pair kp) at (rb * cols/128 + kp) *
+//           4096, half h = K step 2 kp + h;
+//   B side: block (row-block pair rbp, K step ks) at (rbp * cols/64 + ks) *
+//           4096, half h = row block 2 rbp + h.
+// Byte offset of the copy for lane quarter q of the scale of (row r, group b).
+__device__ __forceinline__ int64_t sf_mma_offset(int64_t r, int64_t b, int64_t cols, bool b_side, int q)
 {
     const int64_t rb = r >> 7, rr = r & 127, ks = b >> 2, j = b & 3;
-    return ((rb * (cols / 64) + ks) << 9) + ((rr & 31) << 4) + ((rr >> 5) << 2) + j;
+    const int64_t l = 32 * q + (rr & 31), byte = ((rr >> 5) << 2) + j;
+    const int64_t blk = b_side ? ((rb >> 1) * (cols / 64) + ks) : (rb * (cols / 128) + (ks >> 1));
+    const int64_t h = b_side ? (rb & 1) : (ks & 1);
+    return (blk << 12) + ((l >> 3) << 8) + (h << 7) + ((l & 7) << 4) + byte;
 }
 
 __global__ void __launch_bounds__(256) quant_kernel(const uint16_t *__restrict__ in, int64_t rows, int64_t cols,
                                                     int64_t ld, const float *__restrict__ amax,
-                                                    uint8_t *__restrict__ q, uint8_t *__restrict__ sf, bool sf_mma,
+                                                    uint8_t *__restrict__ q, uint8_t *__restrict__ sf, int sf_layout,
                                                     float *__restrict__ s_g_out)
 {
     const float s_g = tensor_scale(*amax);
@@ -100,13 +111,18 @@ __global__ void __launch_bounds__(256) quant_kernel(const uint16_t *__restrict__
         out = make_uint2(e2m1x8(v), e2m1x8(v + 8));
     }
     *reinterpret_cast<uint2 *>(q + r * (cols / 2) + 8 * b) = out;
-    sf[sf_mma ? sf_mma_offset(r, b, cols) : r * nb + b] = (uint8_t)code;
+    if (sf_layout == 0) {
+        sf[r * nb + b] = (uint8_t)code;
+    } else {
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq) sf[sf_mma_offset(r, b, cols, sf_layout == 2, qq)] = (uint8_t)code;
+    }
 }
 
 }  // namespace nvfp4
 
 int launch_quant_nvfp4(const uint16_t *in, int64_t rows, int64_t cols, int64_t ld, uint8_t *q, uint8_t *sf,
-                       bool sf_mma, float *amax, float *s_g, int sms, cudaStream_t s)
+                       int sf_layout, float *amax, float *s_g, int sms, cudaStream_t s)
 {
     if (cudaMemsetAsync(amax, 0, sizeof(float), s) != cudaSuccess) return MOE_ERR_CUDA;
     if (rows > 0) {
@@ -118,7 +134,7 @@ int launch_quant_nvfp4(const uint16_t *in, int64_t rows, int64_t cols, int64_t l
     }
     const int64_t blocks = rows * (cols / 16);
     nvfp4::quant_kernel<<<(unsigned)((blocks + 255) / 256 > 0 ? (blocks + 255) / 256 : 1), 256, 0, s>>>(
-        in, rows, cols, ld, amax, q, sf, sf_mma, s_g);
+        in, rows, cols, ld, amax, q, sf, sf_layout, s_g);
     count_launch();
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

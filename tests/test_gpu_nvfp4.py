@@ -54,38 +54,50 @@ def test_quant_nvfp4_matches_oracle(A, orc, name):
     same_bits(host(q), nvfp4.pack(codes), "packed e2m1 codes")
 
 
-def sf_mma_layout(S8):
-    """[rows][cols/16] e4m3 scale codes -> the block-scaled MMA's atom layout
-    (512-byte atoms per 128-row block and 64-column step, K steps of a row
-    block consecutive; row 32 r1 + r0, group j of a step at byte 16 r0 + 4 r1
-    + j), as moe.h states it."""
+def sf_mma_layout(S8, side):
+    """[rows][cols/16] e4m3 scale codes -> the NVFP4 GEMM's A- or B-side layout
+    as moe.h states it: 4096-byte blocks, each scale stored once per TMEM lane
+    quarter; inside a block, lane l, half h, byte 4 r1 + j (row 32 r1 + l % 32
+    of a 128-row block, group j of a 64-column step) at (l >> 3) * 256 + h * 128
+    + (l & 7) * 16 + 4 r1 + j.  A: block (row block, step pair), h = step
+    parity.  B: block (row-block pair, step), h = row-block parity."""
     rows, nb = S8.shape
+    cols = nb * 16
+    out = np.zeros(4 * rows * nb, np.uint8)
     r = np.arange(rows)[:, None]
     b = np.arange(nb)[None, :]
-    rr = r & 127
-    off = ((r >> 7) * (nb // 4) + (b >> 2)) * 512 + (rr & 31) * 16 + (rr >> 5) * 4 + (b & 3)
-    out = np.zeros(rows * nb, np.uint8)
-    out[off.ravel()] = S8.ravel()
+    rb, rr, ks, j = r >> 7, r & 127, b >> 2, b & 3
+    if side == "A":
+        blk, h = rb * (cols // 128) + (ks >> 1), ks & 1
+    else:
+        blk, h = (rb >> 1) * (cols // 64) + ks, rb & 1
+    for q in range(4):
+        lane = 32 * q + (rr & 31)
+        off = blk * 4096 + (lane >> 3) * 256 + h * 128 + (lane & 7) * 16 + (rr >> 5) * 4 + j
+        out[np.broadcast_to(off, S8.shape).ravel()] = S8.ravel()
     return out
 
 
-def test_quant_nvfp4_mma_layout(A, orc):
+@pytest.mark.parametrize("side", ["A", "B"])
+def test_quant_nvfp4_mma_layout(A, orc, side):
     from oracle import nvfp4
     from moe_expert_layer_replay_b200.inputs import to_bf16_bits
     rng = np.random.default_rng(96)
-    x = to_bf16_bits((rng.standard_normal((384, 1024)) * np.exp(rng.uniform(-4, 4, (384, 1)))).astype(np.float32))
-    q = torch.empty(384, 512, dtype=torch.uint8, device="cuda")
-    sf = torch.full((384 * 64,), 0xAA, dtype=torch.uint8, device="cuda")
+    rows, cols = 512, 1024
+    x = to_bf16_bits((rng.standard_normal((rows, cols)) * np.exp(rng.uniform(-4, 4, (rows, 1)))).astype(np.float32))
+    q = torch.empty(rows, cols // 2, dtype=torch.uint8, device="cuda")
+    sf = torch.full((4 * rows * cols // 16,), 0xAA, dtype=torch.uint8, device="cuda")
     amax = torch.empty(1, device="cuda")
     s_g = torch.empty(1, device="cuda")
-    A.quant_nvfp4(dev(x), 384, 1024, 1024, q, sf, amax, s_g, sf_layout=A.NVFP4_SF_MMA)
+    layout = A.NVFP4_SF_MMA_A if side == "A" else A.NVFP4_SF_MMA_B
+    A.quant_nvfp4(dev(x), rows, cols, cols, q, sf, amax, s_g, sf_layout=layout)
     torch.cuda.synchronize()
     codes, S8, sg = nvfp4.quant(x)
-    same_bits(host(sf), sf_mma_layout(S8), "e4m3 block scales, MMA layout")
+    same_bits(host(sf), sf_mma_layout(S8, side), f"e4m3 block scales, {side}-side MMA layout")
     same_bits(host(q), nvfp4.pack(codes), "packed e2m1 codes")
     same_bits(host(s_g), np.array([sg], np.float32), "tensor scale")
-    with pytest.raises(A.MoeError):   # the MMA layout needs whole 128-row blocks
-        A.quant_nvfp4(dev(x[:200]), 200, 1024, 1024, q, sf, amax, s_g, sf_layout=A.NVFP4_SF_MMA)
+    with pytest.raises(A.MoeError):   # the MMA layouts need whole 128-row (A) / 256-row (B) blocks
+        A.quant_nvfp4(dev(x[:200]), 200, cols, cols, q, sf, amax, s_g, sf_layout=layout)
 
 
 # segment row counts (multiples of 128, 0 = an empty segment), N, K
@@ -117,17 +129,17 @@ def test_gemm_nvfp4_matches_oracle(A, orc, case):
     x[offs[-1]:] = 0
     W = to_bf16_bits((rng.standard_normal((E, N, K)) * 0.02).astype(np.float32))
     aq = torch.empty(R, K // 2, dtype=torch.uint8, device="cuda")
-    asf = torch.empty(R * K // 16, dtype=torch.uint8, device="cuda")
+    asf = torch.empty(4 * R * K // 16, dtype=torch.uint8, device="cuda")
     amax = torch.empty(1, device="cuda")
     a_sg = torch.empty(1, device="cuda")
-    A.quant_nvfp4(dev(x), R, K, K, aq, asf, amax, a_sg, sf_layout=A.NVFP4_SF_MMA)
+    A.quant_nvfp4(dev(x), R, K, K, aq, asf, amax, a_sg, sf_layout=A.NVFP4_SF_MMA_A)
     bq = torch.empty(E, N, K // 2, dtype=torch.uint8, device="cuda")
-    bsf = torch.empty(E, N * K // 16, dtype=torch.uint8, device="cuda")
+    bsf = torch.empty(E, 4 * N * K // 16, dtype=torch.uint8, device="cuda")
     bamax = torch.empty(E, device="cuda")
     b_sg = torch.empty(E, device="cuda")
     Wd = dev(W)
     for e in range(E):
-        A.quant_nvfp4(Wd[e], N, K, K, bq[e], bsf[e], bamax[e:e + 1], b_sg[e:e + 1], sf_layout=A.NVFP4_SF_MMA)
+        A.quant_nvfp4(Wd[e], N, K, K, bq[e], bsf[e], bamax[e:e + 1], b_sg[e:e + 1], sf_layout=A.NVFP4_SF_MMA_B)
     out = torch.full((R, N), -7.0, dtype=torch.float32, device="cuda")
     A.gemm_nvfp4(R, N, K, E, dev(offs), aq, asf, a_sg, bq, bsf, b_sg, out)
     torch.cuda.synchronize()
