@@ -52,7 +52,7 @@ FP4_OVER_FP8 = 2.0   # nominal dense ratio (9 / 4.5 PFLOP/s): the FP4 peak is th
 # kernel.  Valid only for the kernel sources it was taken on: reported as null
 # as soon as their hash differs.
 GEMM1_TRAFFIC = {
-    "replay": {"sources_sha256_16": "898c98b641d524a5", "bytes": 360.218624e6},
+    "prefill": {"sources_sha256_16": "b5de764488ffcf95", "bytes": 8.83e9 + 2.22e9},
 }
 
 

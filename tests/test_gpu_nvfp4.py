@@ -106,6 +106,7 @@ GEMM_CASES = {
     "grouped_empty_segment": ([128, 0, 384], 512, 768),
     "ffn_shape": ([256, 512, 128, 384], 2048, 2048),
     "deep_k": ([256], 256, 7168),
+    "many_tiles_per_sm": ([2048, 1024, 0, 2048], 2048, 512),   # 320 tiles: 2-3 per persistent CTA
 }
 
 
