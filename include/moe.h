@@ -343,8 +343,9 @@ int moe_grouped_gemm_fp8(int32_t op, const moe_dims *dims, const int32_t *offset
                          const moe_gemm_args *args, void *stream);
 
 /* a4+a6 without the permuted copy of the activations: GATEUP_SILU whose A
- * operand is gathered from the token rows by the GEMM's loads (TMA
- * tile::gather4), so the dispatch writes no R x D FP8 copy.  args->a =
+ * operand is gathered from the token rows by the GEMM's loads (half of each
+ * tile's rows by TMA tile::gather4, half by cp.async), so the dispatch writes
+ * no R x D FP8 copy.  args->a =
  * codes [T][D] and args->sa = scales [D/128][T] of the 1x128 quantisation of
  * x itself (moe_quant_fp8_block(x, T, D, D, 1, 128, ...)); permuted row r
  * is token src_idx[r] / k (src_idx from moe_permute), a row with src_idx < 0

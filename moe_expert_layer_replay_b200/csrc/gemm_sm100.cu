@@ -134,9 +134,10 @@ struct Args {
     float *out_f32;
     int *status;
     uint64_t budget;
-    // gather (a6 only): A rows come from the token-row codes, row r of the
-    // permuted layout being token src_idx[r] / k (no row for src_idx < 0);
-    // row scales sa[kb * T + token]
+    // gather (a6 only): A rows come from the token-row codes a_rows [T][K],
+    // row r of the permuted layout being token src_idx[r] / k (no row for
+    // src_idx < 0); row scales sa[kb * T + token]
+    const uint8_t *a_rows;
     const int32_t *src_idx;
     int k;
     int T;
@@ -232,7 +233,7 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap
 
 // Four rows (row coordinates r0..r3, the same 128-byte column window c0) of a
 // tensor whose map has a one-row box, into four consecutive 128-byte rows of
-// shared memory.
+// shared memory (128-byte swizzled like any TMA tile).
 __device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap *map, int32_t c0, int32_t r0,
                                             int32_t r1, int32_t r2, int32_t r3, uint32_t bar)
 {
@@ -372,7 +373,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     }
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(bar_full + 8 * s, 1);
+            // gathering: the B load's arrival and the 64 gathering threads' cp.async arrivals
+            mbar_init(bar_full + 8 * s, kGather ? 65 : 1);
             mbar_init(bar_empty + 8 * s, 1);
         }
         if (kWgrad)
@@ -415,21 +417,34 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 
     if (warp < EPI_WARP0) {
       asm volatile("setmaxnreg.dec.sync.aligned.u32 40;");
-      if (warp == 0 && kGather) {
-        // ------------------------------------- TMA producer, gathering ----
-        // every lane gathers four A rows (tile rows 4*lane .. 4*lane+3) of
-        // each K block from the token-row codes; lane 0 also loads B
+      if (kGather && (warp == 0 || warp >= 2)) {
+        // ------------------------------------------ producer, gathering ----
+        // The A rows of each K block come from the token-row codes along two
+        // paths at once (each alone kept the tensor core waiting longer): warp 0
+        // loads tile rows 0-63 with TMA tile::gather4 (lanes 0-15, four rows
+        // each) and B with a TMA tile load (lane 0); warps 2-3 copy tile rows
+        // 64-127 with cp.async, one row per thread, 16 bytes a copy, into the
+        // same 128-byte-swizzled layout (a row with no token reads zeros).  The stage's full barrier counts the TMA bytes
+        // and lane 0's arrival plus the 64 threads' cp.async arrivals
+        // (cp.async.mbarrier.arrive.noinc).
+        const bool tma_side = warp == 0;
         int stage = 0;
         uint32_t phase = 0;
         uint32_t pend = 0, pend_phase = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
             const Tile x = tile_of<false>(t, p, offs_s);
-            int tok[4];
+            int tok[4] = {-1, -1, -1, -1};
+            if (tma_side) {
+                if (lane < 16)
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int si = p.src_idx[x.m0 + 4 * lane + i];
-                tok[i] = si >= 0 ? si / p.k : p.T;   // row T is out of range: zeros
+                    for (int i = 0; i < 4; ++i) {
+                        const int si = p.src_idx[x.m0 + 4 * lane + i];
+                        tok[i] = si >= 0 ? si / p.k : p.T;   // row T is out of range: zeros
+                    }
+            } else {
+                const int si = p.src_idx[x.m0 + 64 + 32 * (warp - 2) + lane];
+                tok[0] = si >= 0 ? si / p.k : -1;
             }
             for (int kb = x.kb0; kb < x.kb1; ++kb) {
                 if (!warp_wait_bounded(bar_empty + 8 * stage, phase ^ 1, p.budget, abort_flag, p.status)) {
@@ -439,12 +454,25 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 pend &= ~(1u << stage);
                 const uint32_t fb = bar_full + 8 * stage;
                 const uint32_t dA = sbase + stage * STAGE_BYTES, dB = dA + A_BYTES;
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(fb, STAGE_BYTES);
-                    tma_load_2d(dB, &tmB, kb * BK, x.e * p.N + x.n0, fb);
+                if (tma_side) {
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(fb, L::B_BYTES + A_BYTES / 2);
+                        tma_load_2d(dB, &tmB, kb * BK, x.e * p.N + x.n0, fb);
+                    }
+                    __syncwarp();
+                    if (lane < 16) tma_gather4(dA + 512 * lane, &tmA, kb * BK, tok[0], tok[1], tok[2], tok[3], fb);
+                } else {
+                    const int r = 64 + 32 * (warp - 2) + lane;
+                    const uint8_t *src = tok[0] >= 0 ? p.a_rows + (int64_t)tok[0] * p.K + kb * BK : p.a_rows;
+                    const uint32_t bytes = tok[0] >= 0 ? 16u : 0u;
+#pragma unroll
+                    for (int c = 0; c < BK / 16; ++c)
+                        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(
+                                         dA + r * BK + ((c ^ (r & 7)) << 4)),
+                                     "l"(src + 16 * c), "r"(bytes)
+                                     : "memory");
+                    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(fb) : "memory");
                 }
-                __syncwarp();
-                tma_gather4(dA + 512 * lane, &tmA, kb * BK, tok[0], tok[1], tok[2], tok[3], fb);
                 pend |= 1u << stage;
                 pend_phase = (pend_phase & ~(1u << stage)) | (phase << stage);
                 if (++stage == STAGES) {
@@ -453,7 +481,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 }
             }
         }
-        if (!ok && lane == 0)
+        asm volatile("cp.async.wait_all;" ::: "memory");   // no copy of this thread outlives the CTA
+        if (!ok && tma_side && lane == 0)
             for (int s = 0; s < STAGES; ++s)
                 if (pend & (1u << s)) wait_drain(bar_full + 8 * s, (pend_phase >> s) & 1u);
       } else if (warp == 0) {
@@ -590,6 +619,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                             ok = false;
                             break;
                         }
+                        // (gathering: A was written by cp.async, through the generic
+                        // proxy; the MMA reads it through the async proxy)
+                        if (kGather) fence_proxy_async_smem();
                         tc_fence_after();
                         const uint32_t aA = sbase + stage * STAGE_BYTES, aB = aA + A_BYTES;
                         const uint32_t dtm = tmem_base + (uint32_t)(buf * BN);
@@ -1147,7 +1179,8 @@ int launch_grouped_gemm(int op, const moe_dims &d, int64_t R_cap, const int32_t 
 
 // a6 with its A operand gathered from the token rows: codes xq_tok [T][D]
 // (g.a) and 1x128 scales [D/128][T] (g.sa); permuted row r is token
-// src_idx[r] / k.  The tensor map has one-row boxes (tile::gather4).
+// src_idx[r] / k.  The producer gathers half of the A rows with TMA
+// tile::gather4 (the tensor map has one-row boxes) and half with cp.async.
 int launch_gateup_gather(const moe_dims &d, int64_t R_cap, const int32_t *offsets, const int32_t *src_idx,
                          const moe_gemm_args &g, int *status, uint64_t budget, cudaStream_t s)
 {
@@ -1164,6 +1197,7 @@ int launch_gateup_gather(const moe_dims &d, int64_t R_cap, const int32_t *offset
     a.out_bf16 = g.out_bf16;
     a.status = status;
     a.budget = budget;
+    a.a_rows = g.a;
     a.src_idx = src_idx;
     a.k = d.k;
     a.T = d.T;

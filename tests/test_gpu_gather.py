@@ -1,5 +1,5 @@
 """GATEUP_SILU with its A operand gathered from the token rows
-(moe_gateup_gather_fp8, TMA tile::gather4) against the dispatched path
+(moe_gateup_gather_fp8: TMA tile::gather4 and cp.async) against the dispatched path
 (moe_permute's FP8 dispatch, then moe_grouped_gemm_fp8): the A tile holds the
 same bytes either way (1x128 quantisation is row-local, so a dispatched row
 is its token's row), so h, its codes and scales must be bit-identical; and
