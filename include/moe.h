@@ -325,6 +325,9 @@ enum {
  * WGRAD_GATEUP: a = dGUqT [2I][R_cap], sa = dGUsT [R_cap/128][2I];
  *               b = xqT [D][R_cap], sb = xsT [R_cap/128][D];
  *               out_f32 = dWgu [E][2I][D] fp32 (interleaved rows), +=.
+ * The WGRAD ops add into dW with fp32 reductions in L2 (round to nearest;
+ * a subnormal sum may be flushed to zero); each element gets one add per
+ * call, so the result does not depend on timing.
  * All code/matrix pointers must be 16-byte aligned; for the WGRAD ops the
  * scale arrays sa and sb too. */
 typedef struct {

@@ -996,18 +996,18 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     p.out_s[(int64_t)(2 * nb + 1) * p.R_cap + r] = sus;
                 }
             } else {  // EPI_WGRAD: dW[e][m][n] += acc
+                // The adds run in L2 (vector reductions, no value comes back), so
+                // the next tile's K loop starts without waiting for dW to arrive.
+                // One CTA owns each dW tile, so every element gets exactly one add
+                // per launch: the result does not depend on timing.
                 const int64_t c0 = (int64_t)x.n0 + 128 * h;
                 if (c0 < p.N) {
                     float *o = p.out_f32 + ((int64_t)x.e * p.M + x.m0 + row) * p.N + c0;
 #pragma unroll
-                    for (int i0 = 0; i0 < 128; i0 += 4) {
-                        float4 v = *reinterpret_cast<float4 *>(o + i0);
-                        v.x += acc[i0];
-                        v.y += acc[i0 + 1];
-                        v.z += acc[i0 + 2];
-                        v.w += acc[i0 + 3];
-                        *reinterpret_cast<float4 *>(o + i0) = v;
-                    }
+                    for (int i0 = 0; i0 < 128; i0 += 4)
+                        asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(o + i0), "f"(acc[i0]),
+                                     "f"(acc[i0 + 1]), "f"(acc[i0 + 2]), "f"(acc[i0 + 3])
+                                     : "memory");
                 }
             }
         }
