@@ -329,7 +329,8 @@ enum {
  * a subnormal sum may be flushed to zero); each element gets one add per
  * call, so the result does not depend on timing.
  * All code/matrix pointers must be 16-byte aligned; for the WGRAD ops the
- * scale arrays sa and sb too. */
+ * scale arrays sa and sb too; for DGRAD_DOWN_SILU, aux, out_bf16 and out_q
+ * 32-byte aligned. */
 typedef struct {
     const uint8_t *a;
     const float *sa;

@@ -315,6 +315,21 @@ __device__ __forceinline__ Tile tile_of(int t, const Args &p, const int *offs_s,
     return x;
 }
 
+// 32-byte global accesses (sm_100 vector width); the address must be 32-byte aligned.
+__device__ __forceinline__ void ld_global_32B(const void *src, uint4 *v)
+{
+    asm volatile("ld.global.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(v[0].x), "=r"(v[0].y), "=r"(v[0].z), "=r"(v[0].w), "=r"(v[1].x), "=r"(v[1].y), "=r"(v[1].z),
+                   "=r"(v[1].w)
+                 : "l"(src));
+}
+__device__ __forceinline__ void st_global_32B(void *dst, const uint4 &a, const uint4 &b)
+{
+    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(a.x), "r"(a.y), "r"(a.z),
+                 "r"(a.w), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w)
+                 : "memory");
+}
+
 // --------------------------------------------------------------- kernel ----
 template <int kEpi, bool kGather = false, bool kPair = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -946,51 +961,63 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 // interleaved 2I space are gc = 2nb*128 and uc = gc + 128.
                 //   dg = dH u s (1 + g (1 - s)), du = dH g s, s = sigmoid(g),
                 // each rounded to bf16, stored, and quantised 1x128 (one block
-                // each).  Two passes in registers, no thread-local arrays (local
-                // memory would miss the L1 left beside this kernel's shared
-                // memory): pass 1 makes dg, du, their bf16 rows and the block
-                // maxima; pass 2 re-reads this thread's own bf16 rows (written in
-                // pass 1; the bf16 output is required for this op) and writes the
-                // codes.
+                // each).  Two fully unrolled passes: pass 1 makes dg, du, stores
+                // their bf16 rows and takes the block maxima, keeping the bf16
+                // pairs in registers (they take the places of the accumulators
+                // they replace); pass 2 makes the codes from those registers.
                 const int nb = 2 * x.nt + h;
                 if (nb * 128 < p.N) {
                     const int64_t N2 = 2 * (int64_t)p.N;
                     const int64_t gc = (int64_t)(2 * nb) * 128, uc = gc + 128;
+                    // 32-byte accesses (each lane reads or writes its own row, so
+                    // a warp's access touches 32 rows: wider pieces mean fewer of
+                    // them)
                     const uint16_t *gu = p.aux + r * N2;
-                    auto grads = [&](int i0, float *dg, float *du) {
-                        float g[8], u[8];
-                        unpack8(*reinterpret_cast<const uint4 *>(gu + gc + i0), g);
-                        unpack8(*reinterpret_cast<const uint4 *>(gu + uc + i0), u);
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const float d = acc[i0 + i];
-                            const float sg = sigmoid_fast(g[i]);
-                            dg[i] = __uint_as_float(bf16_bits_rn(d * u[i] * sg * (1.0f + g[i] * (1.0f - sg))) << 16);
-                            du[i] = __uint_as_float(bf16_bits_rn(d * g[i] * sg) << 16);
-                        }
-                    };
+                    uint16_t *ob = p.out_bf16 + r * N2;
+                    uint8_t *oq = p.out_q + r * N2;
                     float amax_g = 0.0f, amax_u = 0.0f;
+                    uint4 bg[16], bu[16];   // bf16 dg, du of columns 8j .. 8j + 7
 #pragma unroll
-                    for (int i0 = 0; i0 < 128; i0 += 8) {
-                        float dg[8], du[8];
-                        grads(i0, dg, du);
-                        amax_g = absmax8(dg, amax_g);
-                        amax_u = absmax8(du, amax_u);
-                        *reinterpret_cast<uint4 *>(p.out_bf16 + r * N2 + gc + i0) = pack8(dg);
-                        *reinterpret_cast<uint4 *>(p.out_bf16 + r * N2 + uc + i0) = pack8(du);
+                    for (int j = 0; j < 16; j += 2) {
+                        uint4 gw[2], uw[2];
+                        ld_global_32B(gu + gc + 8 * j, gw);
+                        ld_global_32B(gu + uc + 8 * j, uw);
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                            float g[8], u[8], dg[8], du[8];
+                            unpack8(gw[hh], g);
+                            unpack8(uw[hh], u);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                const float d = acc[8 * (j + hh) + i];
+                                const float sg = sigmoid_fast(g[i]);
+                                dg[i] = __uint_as_float(bf16_bits_rn(d * u[i] * sg * (1.0f + g[i] * (1.0f - sg))) << 16);
+                                du[i] = __uint_as_float(bf16_bits_rn(d * g[i] * sg) << 16);
+                            }
+                            amax_g = absmax8(dg, amax_g);
+                            amax_u = absmax8(du, amax_u);
+                            bg[j + hh] = pack8(dg);
+                            bu[j + hh] = pack8(du);
+                        }
+                        st_global_32B(ob + gc + 8 * j, bg[j], bg[j + 1]);
+                        st_global_32B(ob + uc + 8 * j, bu[j], bu[j + 1]);
                     }
                     const float sgs = block_scale(amax_g), sus = block_scale(amax_u);
-                    // a rolled loop: one copy of the quantiser's code, not sixteen
-                    const uint16_t *ob = p.out_bf16 + r * N2;
-#pragma unroll 1
-                    for (int i0 = 0; i0 < 128; i0 += 16) {
-                        float dg[16], du[16];
-                        unpack8(*reinterpret_cast<const uint4 *>(ob + gc + i0), dg);
-                        unpack8(*reinterpret_cast<const uint4 *>(ob + gc + i0 + 8), dg + 8);
-                        unpack8(*reinterpret_cast<const uint4 *>(ob + uc + i0), du);
-                        unpack8(*reinterpret_cast<const uint4 *>(ob + uc + i0 + 8), du + 8);
-                        *reinterpret_cast<uint4 *>(p.out_q + r * N2 + gc + i0) = quant16(dg, sgs);
-                        *reinterpret_cast<uint4 *>(p.out_q + r * N2 + uc + i0) = quant16(du, sus);
+#pragma unroll
+                    for (int j = 0; j < 16; j += 4) {
+                        uint4 cg[2], cu[2];
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                            float dg[16], du[16];
+                            unpack8(bg[j + 2 * hh], dg);
+                            unpack8(bg[j + 2 * hh + 1], dg + 8);
+                            unpack8(bu[j + 2 * hh], du);
+                            unpack8(bu[j + 2 * hh + 1], du + 8);
+                            cg[hh] = quant16(dg, sgs);
+                            cu[hh] = quant16(du, sus);
+                        }
+                        st_global_32B(oq + gc + 8 * j, cg[0], cg[1]);
+                        st_global_32B(oq + uc + 8 * j, cu[0], cu[1]);
                     }
                     p.out_s[(int64_t)(2 * nb) * p.R_cap + r] = sgs;
                     p.out_s[(int64_t)(2 * nb + 1) * p.R_cap + r] = sus;

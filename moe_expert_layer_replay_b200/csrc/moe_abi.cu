@@ -34,6 +34,7 @@ uint64_t g_wait_budget = 0;  // 0 = default
 cudaStream_t as_stream(void *s) { return reinterpret_cast<cudaStream_t>(s); }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned32(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 bool aligned8(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 7u) == 0; }
 
@@ -317,9 +318,9 @@ int check_gemm_args(int32_t op, const moe_gemm_args *g)
     case MOE_GEMM_DGRAD_GATEUP:
         if (!g->out_bf16 || !aligned16(g->out_bf16)) return MOE_ERR_INVALID_ARG;
         break;
-    case MOE_GEMM_DGRAD_DOWN_SILU:
-        if (!g->aux || !g->out_q || !g->out_s || !g->out_bf16 || !aligned16(g->aux) || !aligned16(g->out_q) ||
-            !aligned16(g->out_bf16))
+    case MOE_GEMM_DGRAD_DOWN_SILU:  // the output step moves 32-byte pieces of aux, out_bf16 and out_q
+        if (!g->aux || !g->out_q || !g->out_s || !g->out_bf16 || !aligned32(g->aux) || !aligned32(g->out_q) ||
+            !aligned32(g->out_bf16))
             return MOE_ERR_INVALID_ARG;
         break;
     case MOE_GEMM_WGRAD_DOWN:
