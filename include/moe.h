@@ -329,8 +329,9 @@ enum {
  * a subnormal sum may be flushed to zero); each element gets one add per
  * call, so the result does not depend on timing.
  * All code/matrix pointers must be 16-byte aligned; for the WGRAD ops the
- * scale arrays sa and sb too; for DGRAD_DOWN_SILU, aux, out_bf16 and out_q
- * 32-byte aligned. */
+ * scale arrays sa and sb too; 32-byte aligned: aux and out_bf16 of
+ * GATEUP_SILU, and aux, out_bf16 and out_q of DGRAD_DOWN_SILU (their rows
+ * are written or read in 32-byte pieces). */
 typedef struct {
     const uint8_t *a;
     const float *sa;

@@ -875,10 +875,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 float amax = 0.0f;
 #pragma unroll
                 for (int i0 = 0; i0 < 64; i0 += 8) {
-                    if (p.aux) {
+                    if (p.aux && (i0 & 8) == 0) {   // g and u rows (training), 32-byte pieces
                         uint16_t *gu = const_cast<uint16_t *>(p.aux) + r * p.N + x.n0 + 64 * h + i0;
-                        *reinterpret_cast<uint4 *>(gu) = pack8(&acc[i0]);
-                        *reinterpret_cast<uint4 *>(gu + 128) = pack8(&acc[64 + i0]);
+                        st_global_32B(gu, pack8(&acc[i0]), pack8(&acc[i0 + 8]));
+                        st_global_32B(gu + 128, pack8(&acc[64 + i0]), pack8(&acc[64 + i0 + 8]));
                     }
 #pragma unroll
                     for (int i = i0; i < i0 + 8; ++i) {
@@ -927,7 +927,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 if (p.out_bf16) {
                     uint16_t *hb = p.out_bf16 + r * I + icol;
 #pragma unroll
-                    for (int i0 = 0; i0 < 64; i0 += 8) *reinterpret_cast<uint4 *>(hb + i0) = pack8(&acc[i0]);
+                    for (int i0 = 0; i0 < 64; i0 += 16) st_global_32B(hb + i0, pack8(&acc[i0]), pack8(&acc[i0 + 8]));
                 }
             } else if (kEpi == EPI_BF16) {
                 // 32-column chunks through per-warp smem buffers (two, or one per

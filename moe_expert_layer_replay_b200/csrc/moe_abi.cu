@@ -312,7 +312,8 @@ int check_gemm_args(int32_t op, const moe_gemm_args *g)
     switch (op) {
     case MOE_GEMM_GATEUP_SILU:
         if (!g->out_q || !g->out_s || !aligned16(g->out_q)) return MOE_ERR_INVALID_ARG;
-        if ((g->aux && !aligned16(g->aux)) || (g->out_bf16 && !aligned16(g->out_bf16))) return MOE_ERR_INVALID_ARG;
+        // g, u and h rows leave in 32-byte pieces
+        if ((g->aux && !aligned32(g->aux)) || (g->out_bf16 && !aligned32(g->out_bf16))) return MOE_ERR_INVALID_ARG;
         break;
     case MOE_GEMM_DOWN:
     case MOE_GEMM_DGRAD_GATEUP:

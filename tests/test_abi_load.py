@@ -44,7 +44,7 @@ def test_host_only_calls():
 def test_gemm_operand_contract():
     """Per-op operand requirements of moe_grouped_gemm_fp8 are checked on the
     host, before any device work: the SiLU-backward GEMM needs its bf16 output
-    (its codes are made from it) and 32-byte-aligned aux / outputs, and the wgrad GEMMs need 16-byte-aligned
+    (its codes are made from it), both SiLU GEMMs 32-byte-aligned aux / bf16 outputs, and the wgrad GEMMs need 16-byte-aligned
     scale arrays (they are bulk-copied)."""
     from moe_expert_layer_replay_b200 import abi
     L = abi.lib()
@@ -54,13 +54,14 @@ def test_gemm_operand_contract():
     g = abi.GemmArgs(A, A, A, A, A, A, A, None, None)  # b2 without out_bf16
     assert L.moe_grouped_gemm_fp8(abi.GEMM_DGRAD_DOWN_SILU, ctypes.byref(d), offs, ctypes.byref(g), None) \
         == abi.INVALID_ARG
-    # b2 moves 32-byte pieces of aux, out_bf16 and out_q: each must be 32-byte aligned
-    for i in (4, 5, 7):
-        ptrs = [A] * 8 + [None]
-        ptrs[i] = A + 16
-        g = abi.GemmArgs(*ptrs)
-        assert L.moe_grouped_gemm_fp8(abi.GEMM_DGRAD_DOWN_SILU, ctypes.byref(d), offs, ctypes.byref(g), None) \
-            == abi.INVALID_ARG
+    # a6 (training outputs) and b2 move 32-byte pieces of aux, out_bf16 (and b2's
+    # out_q): each must be 32-byte aligned
+    for op, fields in ((abi.GEMM_DGRAD_DOWN_SILU, (4, 5, 7)), (abi.GEMM_GATEUP_SILU, (4, 7))):
+        for i in fields:
+            ptrs = [A] * 8 + [None]
+            ptrs[i] = A + 16
+            g = abi.GemmArgs(*ptrs)
+            assert L.moe_grouped_gemm_fp8(op, ctypes.byref(d), offs, ctypes.byref(g), None) == abi.INVALID_ARG
     for op in (abi.GEMM_WGRAD_DOWN, abi.GEMM_WGRAD_GATEUP):
         g = abi.GemmArgs(A, A + 4, A, A, None, None, None, None, A)  # sa only 4-byte aligned
         assert L.moe_grouped_gemm_fp8(op, ctypes.byref(d), offs, ctypes.byref(g), None) == abi.INVALID_ARG
