@@ -197,6 +197,8 @@ __global__ void __launch_bounds__(256, 4) quant_rows128_kernel(const uint16_t *_
         cp_async_commit_group();   // (an empty group past the end keeps the count)
     };
     const int64_t G = gridDim.x;
+    // 32-byte code stores need a 32-byte aligned output and row stride
+    const bool wide = ((reinterpret_cast<uintptr_t>(qT) | (uintptr_t)ld_rows) & 31) == 0;
     int slot = 0;
     int32_t rw[4], nxt[4];
     rows_of(blockIdx.x, rw);
@@ -225,11 +227,16 @@ __global__ void __launch_bounds__(256, 4) quant_rows128_kernel(const uint16_t *_
         const float s = block_scale(amax);
         const int64_t gc = c0 + col;
         if (gc < cols) {
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int64_t rr = r0 + part * 32 + h * 16;
-                const uint4 codes = quant16(v + 16 * h, s);
-                if (rr < rows) *reinterpret_cast<uint4 *>(qT + gc * ld_rows + rr) = codes;
+            const int64_t rr = r0 + part * 32;
+            const uint4 q0 = quant16(v, s), q1 = quant16(v + 16, s);
+            uint8_t *dst = qT + gc * ld_rows + rr;
+            if (wide && rr + 32 <= rows) {   // the column's 32 codes in one 32-byte store
+                asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(q0.x),
+                             "r"(q0.y), "r"(q0.z), "r"(q0.w), "r"(q1.x), "r"(q1.y), "r"(q1.z), "r"(q1.w)
+                             : "memory");
+            } else {
+                if (rr < rows) *reinterpret_cast<uint4 *>(dst) = q0;
+                if (rr + 16 < rows) *reinterpret_cast<uint4 *>(dst + 16) = q1;
             }
             if (part == 0) sT[(r0 / 128) * cols + gc] = s;
         }
