@@ -768,13 +768,15 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             for (int kb = x.kb0; kb < x.kb1; ++kb) {
                 const float *d = wscale + wstage * WS_FLOATS;
                 float sa, s0, s1;
+                float sa4[4];   // wgrad: the row scales of this thread's four rows (see below)
                 if (kWgrad) {
                     if (!warp_wait_bounded(bar_sfull + 8 * wstage, wphase, p.budget, abort_flag, p.status)) {
                         ok = false;
                         break;
                     }
-                    sa = d[row];
-                    s0 = s1 = 0.0f;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) sa4[i] = d[32 * q + (lane >> 2) + 8 * i];
+                    sa = s0 = s1 = 0.0f;
                 } else {
                     sa = c_a;
                     s0 = c_a * c_b0;
@@ -812,37 +814,51 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     }
                 };
                 uint32_t rr[64];
+                if (kWgrad) {
+                    // The 16x256b shape, 32 columns of this warp's half at a time,
+                    // lanes 0-15 then 16-31 of its quarter: this thread holds rows
+                    // 32q + lane/4 + 8i (i = 0..3) x the column pairs
+                    // 8j + 2(lane%4), +1, so it needs 32 column scales per K block
+                    // instead of 128 (fewer shared loads).  Each column pair's two
+                    // scales come in one 8-byte shared load (the four lanes of a row
+                    // group read 32 contiguous bytes); the scale products sa * sb[n]
+                    // run on two lanes at once (the same fp32 products as two scalar
+                    // multiplies).
 #pragma unroll
-                for (int g = 0; g < 2; ++g) {
+                    for (int g = 0; g < 4; ++g) {
+                        const uint32_t cb = cbase + 128 * h + 32 * g;
+                        MOE_TMEM_LD_16x256b_X4(cb, rr);
+                        MOE_TMEM_LD_16x256b_X4(cb + (16u << 16), rr + 16);
+                        tmem_wait_ld();
+                        if (g == 3) release();
+                        const float *cs = d + BM + 128 * h + 32 * g + 2 * (lane & 3);
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int c16 = 4 * g + j;
-                        MOE_TMEM_LD16(cbase + col_of(c16 >> 1) + 16 * (c16 & 1), rr + 16 * j);
-                    }
-                    tmem_wait_ld();
-                    if (g == 1) release();
+                        for (int j = 0; j < 4; ++j) {
+                            const float2 c2 = *reinterpret_cast<const float2 *>(cs + 8 * j);
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int c16 = 4 * g + j;
-                        const uint32_t *cur = rr + 16 * j;
-                        if (kWgrad) {
-                            // column scales of this piece: 16-byte shared loads (a slot
-                            // is 1536 B, the column part starts 512 B in); the scale
-                            // products sa * sb[n] on two lanes at once (the same fp32
-                            // products as two scalar multiplies)
-                            const float4 *cs = reinterpret_cast<const float4 *>(d + BM + 128 * h + 16 * c16);
-#pragma unroll
-                            for (int i = 0; i < 16; i += 4) {
-                                const float4 c4 = cs[i >> 2];
-                                float p0, p1, p2, p3;
-                                fmul2(p0, p1, sa, sa, c4.x, c4.y);
-                                fmul2(p2, p3, sa, sa, c4.z, c4.w);
-                                ffma2(acc[16 * c16 + i], acc[16 * c16 + i + 1], __uint_as_float(cur[i]),
-                                      __uint_as_float(cur[i + 1]), p0, p1);
-                                ffma2(acc[16 * c16 + i + 2], acc[16 * c16 + i + 3], __uint_as_float(cur[i + 2]),
-                                      __uint_as_float(cur[i + 3]), p2, p3);
+                            for (int i = 0; i < 4; ++i) {
+                                const uint32_t *cur = rr + 16 * (i >> 1) + 4 * j + 2 * (i & 1);
+                                float p0, p1;
+                                fmul2(p0, p1, sa4[i], sa4[i], c2.x, c2.y);
+                                float *a = acc + 2 * (16 * i + 4 * g + j);
+                                ffma2(a[0], a[1], __uint_as_float(cur[0]), __uint_as_float(cur[1]), p0, p1);
                             }
-                        } else {
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int g = 0; g < 2; ++g) {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const int c16 = 4 * g + j;
+                            MOE_TMEM_LD16(cbase + col_of(c16 >> 1) + 16 * (c16 & 1), rr + 16 * j);
+                        }
+                        tmem_wait_ld();
+                        if (g == 1) release();
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const int c16 = 4 * g + j;
+                            const uint32_t *cur = rr + 16 * j;
                             const float sc = (kEpi == EPI_SILU && c16 >= 4) ? s1 : s0;
 #pragma unroll
                             for (int i = 0; i < 16; i += 2)
@@ -1027,14 +1043,36 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 // the next tile's K loop starts without waiting for dW to arrive.
                 // One CTA owns each dW tile, so every element gets exactly one add
                 // per launch: the result does not depend on timing.
+                // acc[2 (16i + jj) + e] = dW row 32q + lane/4 + 8i, column
+                // 128h + 8jj + 2(lane%4) + e of the tile
                 const int64_t c0 = (int64_t)x.n0 + 128 * h;
+                // Lanes 2l and 2l+1 hold neighbouring column pairs; one exchange
+                // per two column groups gives the even lane four columns of group
+                // 2m and the odd lane four of group 2m+1, each added with one
+                // 16-byte reduction.
                 if (c0 < p.N) {
-                    float *o = p.out_f32 + ((int64_t)x.e * p.M + x.m0 + row) * p.N + c0;
+                    const bool odd = lane & 1;
+                    float *o = p.out_f32 + ((int64_t)x.e * p.M + x.m0 + 32 * q + (lane >> 2)) * p.N + c0 +
+                               2 * (lane & 3) + (odd ? 6 : 0);
+                    const int64_t step = 8 * (int64_t)p.N;   // 8 rows down
 #pragma unroll
-                    for (int i0 = 0; i0 < 128; i0 += 4)
-                        asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(o + i0), "f"(acc[i0]),
-                                     "f"(acc[i0 + 1]), "f"(acc[i0 + 2]), "f"(acc[i0 + 3])
-                                     : "memory");
+                    for (int i = 0; i < 4; ++i, o += step) {
+#pragma unroll
+                        for (int m = 0; m < 8; ++m) {
+                            const float *a = acc + 2 * (16 * i + 2 * m);   // group 2m, then 2m+1
+                            const float s0 = odd ? a[0] : a[2], s1 = odd ? a[1] : a[3];
+                            // (volatile: kept in order with the reductions, so the
+                            // exchanges are not all hoisted ahead of them)
+                            float r0, r1;
+                            asm volatile("shfl.sync.bfly.b32 %0, %1, 1, 0x1f, 0xffffffff;" : "=f"(r0) : "f"(s0));
+                            asm volatile("shfl.sync.bfly.b32 %0, %1, 1, 0x1f, 0xffffffff;" : "=f"(r1) : "f"(s1));
+                            const float v0 = odd ? r0 : a[0], v1 = odd ? r1 : a[1];
+                            const float v2 = odd ? a[2] : r0, v3 = odd ? a[3] : r1;
+                            asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(o + 16 * m), "f"(v0),
+                                         "f"(v1), "f"(v2), "f"(v3)
+                                         : "memory");
+                        }
+                    }
                 }
             }
         }

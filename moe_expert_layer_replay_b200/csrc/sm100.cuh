@@ -188,6 +188,18 @@ __device__ __forceinline__ void mma_commit(uint32_t bar)
           "=r"((r)[12]), "=r"((r)[13]), "=r"((r)[14]), "=r"((r)[15])                                  \
         : "r"(taddr))
 
+// 16 lanes x 32 columns (16x256b shape, 4 repeats): thread t gets, for column
+// group j (columns 8j .. 8j+7), r[4j], r[4j+1] = lane t/4, columns 8j + 2(t%4)
+// and +1; r[4j+2], r[4j+3] = the same columns of lane 8 + t/4.
+#define MOE_TMEM_LD_16x256b_X4(taddr, r)                                                              \
+    asm volatile(                                                                                      \
+        "tcgen05.ld.sync.aligned.16x256b.x4.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"   \
+        "%15}, [%16];"                                                                                 \
+        : "=r"((r)[0]), "=r"((r)[1]), "=r"((r)[2]), "=r"((r)[3]), "=r"((r)[4]), "=r"((r)[5]),         \
+          "=r"((r)[6]), "=r"((r)[7]), "=r"((r)[8]), "=r"((r)[9]), "=r"((r)[10]), "=r"((r)[11]),       \
+          "=r"((r)[12]), "=r"((r)[13]), "=r"((r)[14]), "=r"((r)[15])                                  \
+        : "r"(taddr))
+
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 }  // namespace sm100
