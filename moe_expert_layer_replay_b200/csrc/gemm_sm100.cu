@@ -993,11 +993,20 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     uint8_t *oq = p.out_q + r * N2;
                     float amax_g = 0.0f, amax_u = 0.0f;
                     uint4 bg[16], bu[16];   // bf16 dg, du of columns 8j .. 8j + 7
+                    // g, u loaded two steps ahead of their use (the accesses are
+                    // ordered asm, so a load written after a store stays after it)
+                    uint4 gwb[3][2], uwb[3][2];
+                    ld_global_32B(gu + gc, gwb[0]);
+                    ld_global_32B(gu + uc, uwb[0]);
+                    ld_global_32B(gu + gc + 16, gwb[1]);
+                    ld_global_32B(gu + uc + 16, uwb[1]);
 #pragma unroll
                     for (int j = 0; j < 16; j += 2) {
-                        uint4 gw[2], uw[2];
-                        ld_global_32B(gu + gc + 8 * j, gw);
-                        ld_global_32B(gu + uc + 8 * j, uw);
+                        if (j + 4 < 16) {
+                            ld_global_32B(gu + gc + 8 * (j + 4), gwb[((j >> 1) + 2) % 3]);
+                            ld_global_32B(gu + uc + 8 * (j + 4), uwb[((j >> 1) + 2) % 3]);
+                        }
+                        const uint4 *gw = gwb[(j >> 1) % 3], *uw = uwb[(j >> 1) % 3];
 #pragma unroll
                         for (int hh = 0; hh < 2; ++hh) {
                             float g[8], u[8], dg[8], du[8];
