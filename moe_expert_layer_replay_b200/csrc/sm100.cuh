@@ -236,7 +236,9 @@ inline bool make_map(CUtensorMap *map, const void *base, uint64_t cols, uint64_t
 }
 
 // Row-major [rows][cols] output of 1- or 2-byte elements, boxes of 32 rows x
-// 64 bytes, no swizzle (TMA stores of the SiLU and bf16 epilogues).
+// 64 bytes (TMA stores of the SiLU and bf16 epilogues); 2-byte boxes under the
+// 64-byte swizzle, 1-byte boxes plain (the kernels write the boxes in that
+// layout).
 inline bool make_store_map(CUtensorMap *map, void *base, uint64_t cols, uint64_t rows, int esize)
 {
     auto fn = get_encode_fn();
@@ -247,7 +249,8 @@ inline bool make_store_map(CUtensorMap *map, void *base, uint64_t cols, uint64_t
     cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(map, esize == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base,
                     dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    esize == 2 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
