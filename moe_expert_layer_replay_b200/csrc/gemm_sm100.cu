@@ -17,7 +17,12 @@
 //              multiply by that block's scales (row scale x weight-block
 //              scale; per-column for wgrad) and add into fp32 registers; the
 //              freed TMEM buffer is handed back while the MMA fills the
-//              other.  After the last K block: the fused output step.
+//              other.  After the last K block: the fused output step (TMA
+//              stores of bf16 rows or h codes; 32-byte stores of the
+//              SiLU-backward outputs; L2 reductions into dW for wgrad).
+//              Rows mode reads TMEM in the 32x32b shape (a thread = a row),
+//              wgrad in the 16x256b shape (a thread = 4 rows x 32 columns,
+//              fewer column scales per thread).
 // 2-SM variant (rows mode): clusters of two CTAs on two SMs; the leader issues
 // tcgen05.mma.cta_group::2 with M = 256 (each CTA's own 128 rows of A) and
 // N = 128, each K block as two column halves into separate 128-column TMEM
@@ -778,7 +783,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             }
             for (int kb = x.kb0; kb < x.kb1; ++kb) {
                 const float *d = wscale + wstage * WS_FLOATS;
-                float sa, s0, s1;
+                float s0, s1;   // rows mode: row scale x weight-block scale(s)
                 float sa4[4];   // wgrad: the row scales of this thread's four rows (see below)
                 if (kWgrad) {
                     if (!warp_wait_bounded(bar_sfull + 8 * wstage, wphase, p.budget, abort_flag, p.status)) {
@@ -787,9 +792,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     }
 #pragma unroll
                     for (int i = 0; i < 4; ++i) sa4[i] = d[32 * q + (lane >> 2) + 8 * i];
-                    sa = s0 = s1 = 0.0f;
+                    s0 = s1 = 0.0f;
                 } else {
-                    sa = c_a;
                     s0 = c_a * c_b0;
                     s1 = c_a * c_b1;
                     c_a = n_a, c_b0 = n_b0, c_b1 = n_b1;
